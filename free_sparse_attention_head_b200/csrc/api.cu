@@ -1,0 +1,66 @@
+// api.cu -- status strings, version, plan sizing and the tensor-map encoder
+// shared by the kernels' host code.
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+
+namespace svoo {
+
+CUresult encode_tiled_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                         uint32_t box_rows, uint32_t box_cols) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return CUDA_ERROR_NOT_FOUND;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+}  // namespace svoo
+
+using namespace svoo;
+
+extern "C" const char* svoo_status_string(svoo_status s) {
+  switch (s) {
+    case SVOO_OK: return "ok";
+    case SVOO_ERR_INVALID_ARG: return "invalid argument";
+    case SVOO_ERR_WORKSPACE: return "workspace too small";
+    case SVOO_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SVOO_ERR_CUDA: return "CUDA launch or runtime error";
+    case SVOO_ERR_TIMEOUT: return "device wait timed out";
+    case SVOO_ERR_INTERNAL: return "internal error";
+  }
+  return "unknown status";
+}
+
+extern "C" int svoo_version(void) { return (0 << 16) | 1; }
+
+extern "C" svoo_status svoo_plan_counts(const svoo_shape* shape, int n_qc, int n_kc, int block_q,
+                                        int64_t counts[10]) {
+  if (!shape_ok(shape) || !counts) return SVOO_ERR_INVALID_ARG;
+  if (n_qc < 1 || n_qc > 256 || n_kc < 1 || n_kc > 256) return SVOO_ERR_INVALID_ARG;
+  if (block_q != 64 && block_q != 128) return SVOO_ERR_INVALID_ARG;
+  const int64_t BH = bh_of(shape), N = shape->N;
+  const int64_t Gq = groups_q(shape, n_qc), Gk = groups_k(shape, n_kc), W = mask_words(shape, n_kc);
+  counts[0] = BH * Gq * W;                              // kmask (uint64)
+  counts[1] = BH * N;                                   // q_label
+  counts[2] = BH * Gq;                                  // q_sizes
+  counts[3] = BH * 8;                                   // stats
+  counts[4] = BH * N;                                   // q_perm
+  counts[5] = BH * (Gq + 1);                            // q_off
+  counts[6] = BH * N;                                   // k_perm
+  counts[7] = BH * (Gk + 1);                            // k_off
+  counts[8] = BH * tile_cap(shape, n_qc, block_q) * 4;  // tiles
+  counts[9] = BH;                                       // tile_count
+  return SVOO_OK;
+}

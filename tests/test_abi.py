@@ -1,0 +1,107 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every entry point
+that include/svoo.h declares, and rejects bad arguments on the host before any
+launch (these calls never reach the device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import free_sparse_attention_head_b200 as svoo
+from free_sparse_attention_head_b200 import build as svoo_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "svoo.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    svoo_build.build()
+    return svoo.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(svoo_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared()
+    for n in ("svoo_cluster", "svoo_build_mask", "svoo_permute", "svoo_sparse_attn"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = os.popen(f"nm -D --defined-only {svoo.lib_path()}").read()
+    exported = set(re.findall(r"\bT (svoo_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    assert set(svoo.EXPORTS) <= exported
+
+
+def test_status_strings_and_version(lib):
+    assert lib.svoo_status_string(0) == b"ok"
+    assert lib.svoo_status_string(2) == b"workspace too small"
+    assert lib.svoo_version() >= 1
+
+
+def _shape(B=1, H=2, N=1024, d=64, n_text=0):
+    return svoo.Shape(B, H, N, d, n_text)
+
+
+def test_plan_counts(lib):
+    sh = _shape(N=1000, d=128, n_text=24)
+    counts = (ctypes.c_int64 * 10)()
+    assert lib.svoo_plan_counts(ctypes.byref(sh), 16, 70, 64, counts) == 0
+    Gq, Gk = 17, 71
+    W = (Gk + 63) // 64
+    cap = (1000 + 63) // 64 + Gq
+    assert list(counts) == [2 * Gq * W, 2000, 2 * Gq, 16, 2000, 2 * (Gq + 1), 2000, 2 * (Gk + 1),
+                            2 * cap * 4, 2]
+
+
+@pytest.mark.parametrize("bad", [
+    dict(d=96), dict(N=0), dict(B=0), dict(n_text=-1), dict(N=10, n_text=10),
+    dict(B=70000, H=1), dict(H=65536),
+])
+def test_bad_shapes_rejected(lib, bad):
+    sh = _shape(**bad)
+    counts = (ctypes.c_int64 * 10)()
+    assert lib.svoo_plan_counts(ctypes.byref(sh), 16, 16, 64, counts) == 1
+    assert lib.svoo_cluster_workspace_size(ctypes.byref(sh), 16, 16) == 0
+
+
+def test_compute_entry_points_validate_before_launch(lib):
+    sh = _shape()
+    P = ctypes.c_void_p
+    fake = P(0x1000)   # never dereferenced: validation fails first
+    odd = P(0x1001)    # misaligned
+    ws = lib.svoo_cluster_workspace_size(ctypes.byref(sh), 16, 16)
+    assert ws > 0
+    # null inputs
+    assert lib.svoo_cluster(ctypes.byref(sh), None, fake, 16, 16, 10, 0, fake, fake, fake, fake, fake,
+                            fake, fake, ws, None, None) == 1
+    # cluster counts out of range, iters < 1, bad warm flag
+    for nq, nk, it, warm in [(0, 16, 10, 0), (16, 300, 10, 0), (16, 16, 0, 0), (16, 16, 1, 2)]:
+        assert lib.svoo_cluster(ctypes.byref(sh), fake, fake, nq, nk, it, warm, fake, fake, fake, fake,
+                                fake, fake, fake, ws, None, None) == 1
+    # misaligned q
+    assert lib.svoo_cluster(ctypes.byref(sh), odd, fake, 16, 16, 10, 0, fake, fake, fake, fake, fake,
+                            fake, fake, ws, None, None) == 1
+    # workspace too small
+    assert lib.svoo_cluster(ctypes.byref(sh), fake, fake, 16, 16, 10, 0, fake, fake, fake, fake, fake,
+                            fake, fake, ws - 1024, None, None) == 2
+    plan = svoo._CPlan(*([0x1000] * 10))
+    mws = lib.svoo_mask_workspace_size(ctypes.byref(sh), 16, 16)
+    args = [ctypes.byref(sh), fake, fake, fake, fake, fake, fake, 16, 16]
+    assert lib.svoo_build_mask(*args, 2, 64, 2, 0.125, ctypes.byref(plan), fake, mws, None, None) == 1
+    assert lib.svoo_build_mask(*args, 0, 96, 2, 0.125, ctypes.byref(plan), fake, mws, None, None) == 1
+    assert lib.svoo_build_mask(*args, 0, 64, 2, -1.0, ctypes.byref(plan), fake, mws, None, None) == 1
+    assert lib.svoo_build_mask(*args, 0, 64, 2, 0.125, ctypes.byref(plan), fake, 8, None, None) == 2
+    assert lib.svoo_permute(ctypes.byref(sh), fake, fake, fake, fake, 16, 16, 64, ctypes.byref(plan),
+                            odd, fake, fake, None, None) == 1
+    assert lib.svoo_sparse_attn(ctypes.byref(sh), fake, fake, fake, ctypes.byref(plan), 16, 16, 64,
+                                float("nan"), fake, None, None) == 1
+    assert lib.svoo_sparse_attn(ctypes.byref(sh), fake, fake, fake, None, 16, 16, 64, 0.125, fake,
+                                None, None) == 1

@@ -1,0 +1,363 @@
+"""GPU parity of every stage of the path against the CPU oracle.
+
+Each GPU stage is fed inputs from the generator or from the oracle (never from
+another GPU stage) and its outputs are compared with the oracle's:
+
+* clustering half-steps: assignments agree on >= 99.9% of tokens and every
+  disagreement sits where the oracle's own fp64 distances are within 1e-4
+  (relative); with full agreement the centroids and sizes are bit-exact;
+* whole clustering (all iterations): >= 99.9% agreement of the final labels;
+* mask + tail merge, permutation, query tiles, gathered copies: bit-exact;
+* attention: max-abs <= 2e-2 and relative Frobenius <= 1e-2 against the
+  fp64 oracle on the same mask, on every row of the small cases and on
+  sampled rows at full size.
+
+The Wan2.1-14B case runs all 40 heads in one call, as the benchmark does, and
+checks sampled heads / rows; other heads receive copies of the sampled heads'
+oracle inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workload
+import free_sparse_attention_head_b200 as svoo
+from free_sparse_attention_head_b200 import build as svoo_build
+
+from _parity import (check_assign, check_attention, dev, from_dev_bf16, gather_by_plan, inject_plan,
+                     oracle_plan_heads, qkv_tensors, ragged_workload, sample_rows, scale_of,
+                     to_dev_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    svoo_build.build()
+    svoo.load()
+
+
+def _cfg(w, mode=0):
+    return svoo.Config(n_qc=w.n_qc, n_kc=w.n_kc, iters=w.iters, block_q=w.block_q, select_mode=mode)
+
+
+def _sub(w, H):
+    """Same workload restricted to the first H heads (the generator is per head)."""
+    import dataclasses
+    return dataclasses.replace(w, H=H)
+
+
+SMALL = {"tiny": workload.get("tiny"), "ragged": ragged_workload(),
+         "wan1.3b-2heads": _sub(workload.get("wan2.1-1.3b"), 2)}
+
+
+def _err_ok(err):
+    svoo.check_device_errors(err)
+
+
+# ----------------------------------------------------------------------------- clustering
+
+
+def _half_step_case(w, heads_checked):
+    q, k, _ = workload.make_qkv(w)
+    BH, nv, d = w.B * w.H, w.n_video, w.d
+    qd, kd, _ = qkv_tensors(q, k, k, w.B, w.H)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # query step, feature space, from the oracle's deterministic start
+    c0 = np.stack([oracle.init_centroids(q[h][:nv], w.n_qc) for h in range(BH)])
+    cent = dev(c0)
+    sizes = torch.zeros(BH, w.n_qc, dtype=torch.int32, device="cuda")
+    asg = torch.empty(BH, nv, dtype=torch.int32, device="cuda")
+    svoo.cluster_step(qd, cent, sizes, asg, n_text=w.n_text, dev_err=err)
+    torch.cuda.synchronize()
+    _err_ok(err)
+    g_asg, g_cent, g_sz = asg.cpu().numpy(), cent.cpu().numpy(), sizes.cpu().numpy()
+    metric_src = {}
+    for h in heads_checked:
+        a, b1, b2 = oracle.assign(q[h][:nv], c0[h], np.eye(d), with_dist=True)
+        c1, s1 = oracle.update(q[h][:nv], a, c0[h])
+        _, ndiff = check_assign(g_asg[h], a, b1, b2, f"{w.name} q-step head {h}")
+        if ndiff == 0:
+            assert np.array_equal(g_cent[h].view(np.uint32), c1.view(np.uint32))
+            assert np.array_equal(g_sz[h], s1)
+        metric_src[h] = (c1, s1)
+    # key step under the metric of the oracle's updated query clusters
+    kc0 = np.stack([oracle.init_centroids(k[h][:nv], w.n_kc) for h in range(BH)])
+    mcent = c0.copy()
+    msz = np.full((BH, w.n_qc), 1, dtype=np.int32)
+    for h, (c1, s1) in metric_src.items():
+        mcent[h], msz[h] = c1, s1
+    kcent = dev(kc0)
+    ksz = torch.zeros(BH, w.n_kc, dtype=torch.int32, device="cuda")
+    kasg = torch.empty(BH, nv, dtype=torch.int32, device="cuda")
+    svoo.cluster_step(kd, kcent, ksz, kasg, metric_cent=dev(mcent), metric_sizes=dev(msz),
+                      n_text=w.n_text, dev_err=err)
+    torch.cuda.synchronize()
+    _err_ok(err)
+    g_kasg, g_kcent, g_ksz = kasg.cpu().numpy(), kcent.cpu().numpy(), ksz.cpu().numpy()
+    for h in heads_checked:
+        M = oracle.metric(mcent[h], msz[h])
+        a, b1, b2 = oracle.assign(k[h][:nv], kc0[h], M, with_dist=True)
+        c1, s1 = oracle.update(k[h][:nv], a, kc0[h])
+        _, ndiff = check_assign(g_kasg[h], a, b1, b2, f"{w.name} k-step head {h}")
+        if ndiff == 0:
+            assert np.array_equal(g_kcent[h].view(np.uint32), c1.view(np.uint32))
+            assert np.array_equal(g_ksz[h], s1)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_cluster_half_steps(name):
+    w = SMALL[name]
+    _half_step_case(w, range(w.B * w.H))
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_cluster_whole(name):
+    w = SMALL[name]
+    q, k, _ = workload.make_qkv(w)
+    qd, kd, _ = qkv_tensors(q, k, k, w.B, w.H)
+    cl = svoo.cluster(qd, kd, _cfg(w), n_text=w.n_text)
+    torch.cuda.synchronize()
+    _err_ok(cl["dev_err"])
+    nv = w.n_video
+    for h in range(w.B * w.H):
+        o = oracle.cluster(q[h][:nv], k[h][:nv], w.n_qc, w.n_kc, w.iters)
+        for side in ("q", "k"):
+            g = cl[f"{side}_assign"][h].cpu().numpy()
+            agree = (g == o[f"{side}_assign"]).mean()
+            assert agree >= 0.999, (name, h, side, agree)
+            if agree == 1.0:
+                assert np.array_equal(cl[f"{side}_cent"][h].cpu().numpy(), o[f"{side}_cent"])
+                assert np.array_equal(cl[f"{side}_sizes"][h].cpu().numpy(), o[f"{side}_sizes"])
+
+
+# ----------------------------------------------------------------------------- mask, permutation
+
+
+def _mask_case(w, plans, src, mode=0, keeps=None):
+    """GPU build_mask on the oracle's clustering of head src[h]; compare with the oracle plan."""
+    BH = len(src)
+    sh = svoo.Shape(1, BH, w.N, w.d, w.n_text)
+    cfg = _cfg(w, mode)
+    cl = dict(
+        q_cent=dev(np.stack([plans[s]["cl"]["q_cent"] for s in src])),
+        k_cent=dev(np.stack([plans[s]["cl"]["k_cent"] for s in src])),
+        q_sizes=dev(np.stack([plans[s]["cl"]["q_sizes"] for s in src])),
+        k_sizes=dev(np.stack([plans[s]["cl"]["k_sizes"] for s in src])),
+        q_assign=dev(np.stack([plans[s]["cl"]["q_assign"] for s in src])),
+    )
+    keep = dev(np.asarray([keeps[s] for s in src], dtype=np.float32))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    plan = svoo.build_mask(sh, cl, keep, cfg, dev_err=err)
+    torch.cuda.synchronize()
+    _err_ok(err)
+    V = plan.views()
+    for h, s in enumerate(src):
+        p = plans[s]
+        assert np.array_equal(V["kmask"][h].cpu().numpy().view(np.uint64), p["kmask"]), (w.name, h)
+        assert np.array_equal(V["q_label"][h].cpu().numpy(), p["q_label"]), (w.name, h)
+        Gq = plan.Gq
+        want_sizes = np.concatenate([p["q_sizes_merged"], [w.n_text]]) if w.n_text else p["q_sizes_merged"]
+        assert np.array_equal(V["q_sizes"][h].cpu().numpy(), want_sizes[:Gq])
+        st = V["stats"][h].cpu().numpy()
+        ms = p["merge_stats"]
+        assert st.tolist() == [p["kept"], p["nonempty"], ms[0], ms[1], ms[2], ms[3], ms[4], ms[5]], (w.name, h)
+    return plan
+
+
+def _keeps(w, mode):
+    if mode == 0:
+        return w.keep_ratios()
+    return np.linspace(0.5, 0.95, w.B * w.H).astype(np.float32)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("mode", [0, 1])
+def test_mask_and_tail_merge(name, mode):
+    w = SMALL[name]
+    q, k, _ = workload.make_qkv(w)
+    keeps = _keeps(w, mode)
+    heads = list(range(w.B * w.H))
+    plans = oracle_plan_heads(w, q, k, heads, keeps, mode=mode)
+    _mask_case(w, plans, heads, mode, keeps)
+
+
+def _permute_case(w, q, k, v, plans, src):
+    BH = len(src)
+    sh = svoo.Shape(1, BH, w.N, w.d, w.n_text)
+    plan = svoo.Plan(sh, _cfg(w), "cuda")
+    inject_plan(plan, plans, src)
+    V = plan.views()
+    # clear what permute must produce
+    for f in ("q_perm", "q_off", "k_perm", "k_off", "tiles", "tile_count"):
+        V[f].fill_(-7)
+    k_assign = dev(np.stack([plans[s]["k_label"][:w.n_video] for s in src]))
+    qd, kd, vd = qkv_tensors(q, k, v, 1, BH)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qp, kp, vp = svoo.permute(qd, kd, vd, k_assign, plan, dev_err=err)
+    torch.cuda.synchronize()
+    _err_ok(err)
+    V = plan.views()
+    eq, ek, ev = gather_by_plan(q, k, v, plans, src)
+    assert np.array_equal(from_dev_bf16(qp).reshape(eq.shape), eq)
+    assert np.array_equal(from_dev_bf16(kp).reshape(ek.shape), ek)
+    assert np.array_equal(from_dev_bf16(vp).reshape(ev.shape), ev)
+    ref = svoo.Plan(sh, _cfg(w), "cuda")
+    inject_plan(ref, plans, src)
+    R = ref.views()
+    for f in ("q_perm", "q_off", "k_perm", "k_off", "tiles", "tile_count"):
+        assert torch.equal(V[f], R[f]), (w.name, f)
+    return plan, qp, kp, vp
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_permute_tiles_gather(name):
+    w = SMALL[name]
+    q, k, v = workload.make_qkv(w)
+    heads = list(range(w.B * w.H))
+    plans = oracle_plan_heads(w, q, k, heads, w.keep_ratios())
+    _permute_case(w, q, k, v, plans, heads)
+
+
+# ----------------------------------------------------------------------------- attention
+
+
+def _attn_case(w, q, k, v, plans, src, rows_per_head, heads_checked, seed=0):
+    BH = len(src)
+    sh = svoo.Shape(1, BH, w.N, w.d, w.n_text)
+    plan = svoo.Plan(sh, _cfg(w), "cuda")
+    inject_plan(plan, plans, src)
+    eq, ek, ev = gather_by_plan(q, k, v, plans, src)
+    qp, kp, vp = qkv_tensors(eq, ek, ev, 1, BH)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = svoo.sparse_attn(qp, kp, vp, plan, dev_err=err)
+    torch.cuda.synchronize()
+    _err_ok(err)
+    o = from_dev_bf16(out).reshape(BH, w.N, w.d)
+    scale = scale_of(w.d)
+    worst = (0.0, 0.0)
+    for h in heads_checked:
+        p = plans[src[h]]
+        rows = sample_rows(w.N, rows_per_head, seed + h)
+        ref, psum, nk = oracle.attn_rows(q[h], k[h], v[h], scale, p["q_label"], p["k_label"], p["kmask"], rows)
+        ma, fr = check_attention(o[h][rows], ref, f"{w.name} head {h}")
+        worst = (max(worst[0], ma), max(worst[1], fr))
+    return worst
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_attention(name):
+    w = SMALL[name]
+    q, k, v = workload.make_qkv(w)
+    heads = list(range(w.B * w.H))
+    plans = oracle_plan_heads(w, q, k, heads, w.keep_ratios())
+    rows = w.N if w.N <= 2048 else 1024
+    _attn_case(w, q, k, v, plans, heads, rows, heads)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_dense_keep_one_equals_dense_attention(name):
+    """keep = 1.0: the sparse kernel over every tile equals textbook attention."""
+    w = SMALL[name]
+    q, k, v = workload.make_qkv(w)
+    heads = list(range(w.B * w.H))
+    keeps = np.ones(len(heads), dtype=np.float32)
+    plans = oracle_plan_heads(w, q, k, heads, keeps)
+    BH = len(heads)
+    sh = svoo.Shape(1, BH, w.N, w.d, w.n_text)
+    plan = svoo.Plan(sh, _cfg(w), "cuda")
+    inject_plan(plan, plans, heads)
+    eq, ek, ev = gather_by_plan(q, k, v, plans, heads)
+    qp, kp, vp = qkv_tensors(eq, ek, ev, 1, BH)
+    out = svoo.sparse_attn(qp, kp, vp, plan)
+    o = from_dev_bf16(out).reshape(BH, w.N, w.d)
+    for h in heads:
+        rows = sample_rows(w.N, 512, h)
+        ref = oracle.dense_attn_rows(q[h], k[h], v[h], scale_of(w.d), rows)
+        check_attention(o[h][rows], ref, f"dense {name} head {h}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_end_to_end_small(name):
+    """The whole GPU path from Q, K, V; where the clustering agrees with the
+    oracle exactly, the plan must be bit-exact and O within tolerance."""
+    w = SMALL[name]
+    q, k, v = workload.make_qkv(w)
+    qd, kd, vd = qkv_tensors(q, k, v, w.B, w.H)
+    keep = dev(w.keep_ratios())
+    out, st = svoo.sparse_attention(qd, kd, vd, keep, _cfg(w), n_text=w.n_text)
+    torch.cuda.synchronize()
+    _err_ok(st["dev_err"])
+    o = from_dev_bf16(out).reshape(w.B * w.H, w.N, w.d)
+    V = st["plan"].views()
+    heads = list(range(w.B * w.H))
+    plans = oracle_plan_heads(w, q, k, heads, w.keep_ratios())
+    for h in heads:
+        p = plans[h]
+        same = np.array_equal(st["cl"]["q_assign"][h].cpu().numpy(), p["cl"]["q_assign"]) and \
+            np.array_equal(st["cl"]["k_assign"][h].cpu().numpy(), p["cl"]["k_assign"])
+        assert same, f"{name} head {h}: clustering differs from the oracle"
+        assert np.array_equal(V["kmask"][h].cpu().numpy().view(np.uint64), p["kmask"])
+        assert np.array_equal(V["q_perm"][h].cpu().numpy(), p["q_perm"])
+        rows = np.arange(w.N, dtype=np.int32)
+        ref, _, _ = oracle.attn_rows(q[h], k[h], v[h], scale_of(w.d), p["q_label"], p["k_label"],
+                                     p["kmask"], rows)
+        check_attention(o[h], ref, f"e2e {name} head {h}")
+
+
+# ----------------------------------------------------------------------------- full sizes
+
+
+def test_wan14b_full_size():
+    """All 40 heads at the Wan2.1-14B shape in one launch (the benchmark's
+    configuration); sampled heads checked stage by stage against the oracle,
+    and invariants of the GPU's own end-to-end plan checked on every head."""
+    w = workload.get("wan2.1-14b")
+    q, k, v = workload.make_qkv(w)
+    BH = w.B * w.H
+    sampled = [0, 37]
+    _half_step_case(w, sampled)
+    keeps = w.keep_ratios()
+    plans = oracle_plan_heads(w, q[sampled], k[sampled], [0, 1], keeps[sampled], iters=2)
+    src = [h % 2 for h in range(BH)]
+    # masks: oracle inputs of the sampled heads, copied to every head
+    _mask_case(w, plans, src, 0, {i: keeps[sampled[i]] for i in range(2)})
+    qs = np.stack([q[sampled[s]] for s in src])
+    ks = np.stack([k[sampled[s]] for s in src])
+    vs = np.stack([v[sampled[s]] for s in src])
+    _permute_case(w, qs, ks, vs, plans, src)
+    _attn_case(w, qs, ks, vs, plans, src, 768, [0, 1, 39])
+    # end to end on the real 40-head input: invariants on every head
+    qd, kd, vd = qkv_tensors(q, k, v, w.B, w.H)
+    out, st = svoo.sparse_attention(qd, kd, vd, dev(keeps), _cfg(w))
+    torch.cuda.synchronize()
+    _err_ok(st["dev_err"])
+    assert torch.isfinite(out.float()).all()
+    V = st["plan"].views()
+    N = w.N
+    P = w.n_qc * w.n_kc
+    for h in range(BH):
+        perm = V["q_perm"][h].cpu().numpy()
+        assert np.array_equal(np.sort(perm), np.arange(N))
+        kperm = V["k_perm"][h].cpu().numpy()
+        assert np.array_equal(np.sort(kperm), np.arange(N))
+        K = math.ceil(np.float32(keeps[h]) * np.float32(P))
+        assert V["stats"][h][0].item() == max(K, w.n_qc)
+        tiles = V["tiles"][h][: V["tile_count"][h].item()].cpu().numpy()
+        assert tiles[:, 2].sum() == N and tiles[:, 2].max() <= w.block_q
+        assert st["cl"]["q_sizes"][h].sum().item() == N and st["cl"]["k_sizes"][h].sum().item() == N
+
+
+def test_hunyuan_text_tokens():
+    """HunyuanVideo shape with 256 always-kept text tokens (2 heads)."""
+    w = _sub(workload.get("hunyuanvideo-13b"), 2)
+    q, k, v = workload.make_qkv(w)
+    heads = [0, 1]
+    keeps = w.keep_ratios(t=10)
+    plans = oracle_plan_heads(w, q, k, heads, keeps, iters=2)
+    _mask_case(w, plans, heads, 0, keeps)
+    _permute_case(w, q, k, v, plans, heads)
+    _attn_case(w, q, k, v, plans, heads, 512, heads)
