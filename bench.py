@@ -224,6 +224,8 @@ def run_gpu(args):
     w = workload.get(WORKLOAD)
     import dataclasses
     w = dataclasses.replace(w, seed=w.seed + rank)  # this rank's own batch element
+    if args.heads:
+        w = dataclasses.replace(w, H=args.heads)
     q, k, v = workload.make_qkv(w)
     BH, N, d = w.B * w.H, w.N, w.d
 
@@ -382,6 +384,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="svoo", choices=["svoo", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the first H heads only (smaller profiling captures; not a bench line)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -5,12 +5,12 @@
 // cold first query step).
 //
 // Kernels of one half-step (one side):
-//   metric_m_kernel      M from the other side's centroids and sizes (fp32)
-//   metric_nu_kernel     nu_j = M mu_j, kappa_j = mu_j . nu_j, |nu_j|, bf16(nu_j)
+//   metric_m_kernel      M from the other side's centroids and sizes (fp64)
+//   metric_nu_kernel     nu_j = M mu_j, kappa_j = mu_j . nu_j (fp64), |nu_j|, bf16(nu_j)
 //   assign_update_kernel tcgen05 bf16 MMA of a 128-token tile against all
 //                        bf16(nu_j) into TMEM; per token the score
 //                        kappa_j - 2 x.nu_j is bounded by the MMA error, every
-//                        candidate that can still win is re-evaluated in fp32
+//                        candidate that can still win is re-evaluated in fp64
 //                        and the argmin (ties to the smaller j) is the label;
 //                        then the tile's tokens are sorted by label and each
 //                        label run is summed in fp64 and added atomically
@@ -41,67 +41,67 @@ __global__ void init_centroids_kernel(const uint16_t* __restrict__ x, int N, int
 
 // ---------------------------------------------------------------- metric
 
-// M[h] = sum_b n_b c_b c_b^T / sum_b n_b. grid (d/8, BH), block d threads;
-// thread j owns column j of rows i0..i0+7.
+// M[h] = sum_b n_b c_b c_b^T / sum_b n_b in fp64. grid (d/8, BH), block d
+// threads; thread j owns column j of rows i0..i0+7.
 __global__ void metric_m_kernel(const float* __restrict__ cent, const int32_t* __restrict__ sizes,
-                                int C, int d, float* __restrict__ M) {
-  extern __shared__ float sm_m[];  // [32][d] centroid chunk, then [32] sizes
-  float* cch = sm_m;
-  float* nch = sm_m + 32 * d;
+                                int C, int d, double* __restrict__ M) {
+  extern __shared__ double sm_m[];  // [32][d] centroid chunk, then [32] sizes
+  double* cch = sm_m;
+  double* nch = sm_m + 32 * d;
   const int h = blockIdx.y, i0 = blockIdx.x * 8, j = threadIdx.x;
-  float acc[8];
+  double acc[8];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+  for (int r = 0; r < 8; ++r) acc[r] = 0.0;
   long long total = 0;
   for (int b0 = 0; b0 < C; b0 += 32) {
     int nb = min(32, C - b0);
     __syncthreads();
     for (int e = threadIdx.x; e < nb * d; e += blockDim.x)
-      cch[e] = cent[(static_cast<size_t>(h) * C + b0) * d + e];
-    if (threadIdx.x < nb) nch[threadIdx.x] = static_cast<float>(sizes[h * C + b0 + threadIdx.x]);
+      cch[e] = static_cast<double>(cent[(static_cast<size_t>(h) * C + b0) * d + e]);
+    if (threadIdx.x < nb) nch[threadIdx.x] = static_cast<double>(sizes[h * C + b0 + threadIdx.x]);
     __syncthreads();
     for (int bb = 0; bb < nb; ++bb) {
-      float n = nch[bb];
+      double n = nch[bb];
       total += static_cast<long long>(n);
-      if (n == 0.f) continue;
-      float cj = n * cch[bb * d + j];
+      if (n == 0.0) continue;
+      double cj = n * cch[bb * d + j];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) acc[r] = fmaf(cch[bb * d + i0 + r], cj, acc[r]);
+      for (int r = 0; r < 8; ++r) acc[r] = fma(cch[bb * d + i0 + r], cj, acc[r]);
     }
   }
-  float inv = total > 0 ? 1.0f / static_cast<float>(total) : 0.f;
 #pragma unroll
   for (int r = 0; r < 8; ++r) {
-    float v = total > 0 ? acc[r] * inv : (i0 + r == j ? 1.f : 0.f);
+    double v = total > 0 ? acc[r] / static_cast<double>(total) : (i0 + r == j ? 1.0 : 0.0);
     M[(static_cast<size_t>(h) * d + i0 + r) * d + j] = v;
   }
 }
 
-// nu_j = M mu_j (M symmetric, read by columns), kappa_j = mu_j . nu_j, |nu_j|,
-// bf16(nu_j); clusters j in [C, Cpad) are padding (nu = 0, kappa = +inf).
+// nu_j = M mu_j (M symmetric, read by columns), kappa_j = mu_j . nu_j in fp64;
+// also bf16(nu_j) for the scoring MMA, fp32 kappa and |nu_j| for its error
+// bound. Clusters j in [C, Cpad) are padding (nu = 0, kappa = +inf).
 // grid (Cpad/8, BH), block d threads; M == nullptr means identity.
-__global__ void metric_nu_kernel(const float* __restrict__ M, const float* __restrict__ cent, int C,
-                                 int Cpad, int d, float* __restrict__ nu,
-                                 uint16_t* __restrict__ nu_bf16, float* __restrict__ kappa,
-                                 float* __restrict__ nunorm) {
-  extern __shared__ float sm_nu[];  // [8][d] mu rows, [8][4] reduction scratch x2
-  float* mu = sm_nu;
-  float* red = sm_nu + 8 * d;
+__global__ void metric_nu_kernel(const double* __restrict__ M, const float* __restrict__ cent, int C,
+                                 int Cpad, int d, double* __restrict__ nu64,
+                                 uint16_t* __restrict__ nu_bf16, double* __restrict__ kappa64,
+                                 float* __restrict__ kappa32, float* __restrict__ nunorm) {
+  extern __shared__ double sm_nu[];  // [8][d] mu rows, [8][4][2] reduction scratch
+  double* mu = sm_nu;
+  double* red = sm_nu + 8 * d;
   const int h = blockIdx.y, j0 = blockIdx.x * 8, i = threadIdx.x;
   for (int e = threadIdx.x; e < 8 * d; e += blockDim.x) {
     int r = e / d, c = e % d;
-    mu[e] = (j0 + r < C) ? cent[(static_cast<size_t>(h) * C + j0 + r) * d + c] : 0.f;
+    mu[e] = (j0 + r < C) ? static_cast<double>(cent[(static_cast<size_t>(h) * C + j0 + r) * d + c]) : 0.0;
   }
   __syncthreads();
-  float acc[8];
+  double acc[8];
   if (M) {
 #pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r] = 0.f;
-    const float* Mh = M + static_cast<size_t>(h) * d * d;
+    for (int r = 0; r < 8; ++r) acc[r] = 0.0;
+    const double* Mh = M + static_cast<size_t>(h) * d * d;
     for (int l = 0; l < d; ++l) {
-      float m = Mh[static_cast<size_t>(l) * d + i];
+      double m = Mh[static_cast<size_t>(l) * d + i];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) acc[r] = fmaf(m, mu[r * d + l], acc[r]);
+      for (int r = 0; r < 8; ++r) acc[r] = fma(m, mu[r * d + l], acc[r]);
     }
   } else {
 #pragma unroll
@@ -112,11 +112,11 @@ __global__ void metric_nu_kernel(const float* __restrict__ M, const float* __res
   for (int r = 0; r < 8; ++r) {
     int j = j0 + r;
     size_t o = (static_cast<size_t>(h) * Cpad + j) * d + i;
-    if (j < C) nu[(static_cast<size_t>(h) * C + j) * d + i] = acc[r];
-    __nv_bfloat16 b = __float2bfloat16_rn(j < C ? acc[r] : 0.f);
+    if (j < C) nu64[(static_cast<size_t>(h) * C + j) * d + i] = acc[r];
+    __nv_bfloat16 b = __float2bfloat16_rn(j < C ? static_cast<float>(acc[r]) : 0.f);
     nu_bf16[o] = *reinterpret_cast<uint16_t*>(&b);
-    float k1 = mu[r * d + i] * acc[r];
-    float k2 = acc[r] * acc[r];
+    double k1 = mu[r * d + i] * acc[r];
+    double k2 = acc[r] * acc[r];
     for (int s = 16; s > 0; s >>= 1) {
       k1 += __shfl_xor_sync(0xffffffffu, k1, s);
       k2 += __shfl_xor_sync(0xffffffffu, k2, s);
@@ -129,13 +129,14 @@ __global__ void metric_nu_kernel(const float* __restrict__ M, const float* __res
   __syncthreads();
   if (threadIdx.x < 8) {
     int r = threadIdx.x, j = j0 + r;
-    float k1 = 0.f, k2 = 0.f;
+    double k1 = 0.0, k2 = 0.0;
     for (int w = 0; w < nwarp; ++w) {
       k1 += red[(r * 4 + w) * 2 + 0];
       k2 += red[(r * 4 + w) * 2 + 1];
     }
-    kappa[h * Cpad + j] = j < C ? k1 : INFINITY;
-    nunorm[h * Cpad + j] = j < C ? sqrtf(k2) : 0.f;
+    kappa64[h * Cpad + j] = j < C ? k1 : INFINITY;
+    kappa32[h * Cpad + j] = j < C ? static_cast<float>(k1) : INFINITY;
+    nunorm[h * Cpad + j] = j < C ? static_cast<float>(sqrt(k2)) : 0.f;
   }
 }
 
@@ -158,8 +159,9 @@ static_assert(sizeof(AssignSmem) <= kAssignHeader, "header overflow");
 __global__ void __launch_bounds__(kAssignThreads)
     assign_update_kernel(const __grid_constant__ CUtensorMap xmap, int N, int nv, int d, int C,
                          int Cpad, int tmem_cols, int tiles_per_cta,
-                         const uint16_t* __restrict__ nu_bf16, const float* __restrict__ nu,
-                         const float* __restrict__ kappa_g, const float* __restrict__ nunorm_g,
+                         const uint16_t* __restrict__ nu_bf16, const double* __restrict__ nu64,
+                         const double* __restrict__ kappa64, const float* __restrict__ kappa_g,
+                         const float* __restrict__ nunorm_g,
                          int32_t* __restrict__ assign, double* __restrict__ sums,
                          int32_t* __restrict__ counts, int* __restrict__ err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -210,7 +212,8 @@ __global__ void __launch_bounds__(kAssignThreads)
 
   const uint32_t idesc = idesc_bf16_f32(128, Cpad, false, false);
   const uint32_t xs_u32 = smem_u32(xs), nus_u32 = smem_u32(nus);
-  const float* nu_h = nu + static_cast<size_t>(h) * C * d;
+  const double* nu_h = nu64 + static_cast<size_t>(h) * C * d;
+  const double* kap64 = kappa64 + static_cast<size_t>(h) * Cpad;
   const size_t xrow0 = static_cast<size_t>(h) * N;
 
   int it = 0;
@@ -286,32 +289,29 @@ __global__ void __launch_bounds__(kAssignThreads)
       }
     }
     tc_fence_before();
+    // Decision: a single candidate is the argmin; otherwise the candidates
+    // are re-scored exactly as the definition reads, kappa_j - 2 x.nu_j in
+    // fp64 (nu, kappa from the fp64 metric), ties to the smaller j.
     int best_j = 0;
-    float best = INFINITY;
-    auto exact_score = [&](int j) {
-      const float* nj = nu_h + static_cast<size_t>(j) * d;
-      float dot = 0.f;
+    auto exact_score = [&](int j) -> double {
+      const double* nj = nu_h + static_cast<size_t>(j) * d;
+      double dot = 0.0;
       for (int c = 0; c < d; ++c) {
         float xv = bf16_to_f32(*reinterpret_cast<const uint16_t*>(xrow + sw128_offset(r, c, kTileRows)));
-        dot = fmaf(xv, __ldg(nj + c), dot);
+        dot = fma(static_cast<double>(xv), __ldg(nj + c), dot);
       }
-      return kap[j] - 2.f * dot;
+      return kap64[j] - 2.0 * dot;
     };
     if (valid) {
-      if (!overflow) {
-        for (int k = 0; k < kMaxCandidates; ++k) {
-          if (k >= ncand) break;
-          int j = cand[k];
-          float s = exact_score(j);
-          if (s < best || (s == best && j < best_j)) {
-            best = s;
-            best_j = j;
-          }
-        }
+      if (ncand == 1) {
+        best_j = cand[0];
       } else {
-        for (int j = 0; j < C; ++j) {
-          float s = exact_score(j);
-          if (s < best) {
+        double best = INFINITY;
+        const int n_eval = overflow ? C : ncand;
+        for (int k = 0; k < n_eval; ++k) {
+          const int j = overflow ? k : cand[k < kMaxCandidates ? k : 0];
+          const double s = exact_score(j);
+          if (s < best) {  // candidates ascend in j: ties keep the smaller j
             best = s;
             best_j = j;
           }
@@ -413,9 +413,10 @@ __global__ void finalize_kernel(double* __restrict__ sums, int32_t* __restrict__
 namespace {
 
 struct StepWs {
-  float* M;
-  float* nu;
+  double* M;
+  double* nu64;
   uint16_t* nu_bf16;
+  double* kappa64;
   float* kappa;
   float* nunorm;
   double* sums;
@@ -424,11 +425,12 @@ struct StepWs {
 
 size_t carve_step(void* ws, int BH, int d, int Cmax, StepWs* out) {
   Carver cv(ws);
-  int Cpad = pad16(Cmax);
+  int Cpad = pad32(Cmax);
   StepWs w;
-  w.M = cv.take<float>(static_cast<size_t>(BH) * d * d);
-  w.nu = cv.take<float>(static_cast<size_t>(BH) * Cmax * d);
+  w.M = cv.take<double>(static_cast<size_t>(BH) * d * d);
+  w.nu64 = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
   w.nu_bf16 = cv.take<uint16_t>(static_cast<size_t>(BH) * Cpad * d);
+  w.kappa64 = cv.take<double>(static_cast<size_t>(BH) * Cpad);
   w.kappa = cv.take<float>(static_cast<size_t>(BH) * Cpad);
   w.nunorm = cv.take<float>(static_cast<size_t>(BH) * Cpad);
   w.sums = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
@@ -454,7 +456,7 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
                      int metric_C, const StepWs& w, int32_t* dev_err, cudaStream_t st,
                      int zero_C) {
   const int BH = bh_of(sh), d = sh->d, N = sh->N, nv = nvideo_of(sh);
-  const int Cpad = pad16(C);
+  const int Cpad = pad32(C);
   // finalize_kernel re-zeroes what a step used, so only the first step of a
   // call clears the accumulators (for the largest cluster count of the call).
   if (zero_C > 0) {
@@ -463,11 +465,11 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
       return SVOO_ERR_CUDA;
   }
   if (metric_cent) {
-    metric_m_kernel<<<dim3(d / 8, BH), d, (32 * d + 32) * sizeof(float), st>>>(metric_cent, metric_sizes,
-                                                                               metric_C, d, w.M);
+    metric_m_kernel<<<dim3(d / 8, BH), d, (32 * d + 32) * sizeof(double), st>>>(metric_cent, metric_sizes,
+                                                                                metric_C, d, w.M);
   }
-  metric_nu_kernel<<<dim3(Cpad / 8, BH), d, (8 * d + 64) * sizeof(float), st>>>(
-      metric_cent ? w.M : nullptr, cent, C, Cpad, d, w.nu, w.nu_bf16, w.kappa, w.nunorm);
+  metric_nu_kernel<<<dim3(Cpad / 8, BH), d, (8 * d + 64) * sizeof(double), st>>>(
+      metric_cent ? w.M : nullptr, cent, C, Cpad, d, w.nu64, w.nu_bf16, w.kappa64, w.kappa, w.nunorm);
   CUtensorMap xmap;
   if (encode_tiled_2d(&xmap, x, static_cast<uint64_t>(BH) * N, d, kTileRows, 64) != CUDA_SUCCESS)
     return SVOO_ERR_CUDA;
@@ -478,7 +480,7 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
                            static_cast<int>(smem)) != cudaSuccess)
     return SVOO_ERR_CUDA;
   assign_update_kernel<<<dim3((ntiles + tpc - 1) / tpc, BH), kAssignThreads, smem, st>>>(
-      xmap, N, nv, d, C, Cpad, tmem_cols_for(Cpad), tpc, w.nu_bf16, w.nu, w.kappa, w.nunorm,
+      xmap, N, nv, d, C, Cpad, tmem_cols_for(Cpad), tpc, w.nu_bf16, w.nu64, w.kappa64, w.kappa, w.nunorm,
       assign, w.sums, w.counts, dev_err);
   finalize_kernel<<<dim3(C, BH), d, 0, st>>>(w.sums, w.counts, cent, sizes, C, d);
   return launch_status();

@@ -50,10 +50,12 @@ def check_assign(gpu_assign, o_assign, best, second, what=""):
     o = np.asarray(o_assign)
     diff = g != o
     agree = 1.0 - diff.mean()
-    assert agree >= ASSIGN_AGREE, f"{what}: agreement {agree:.6f}"
+    gap_max = 0.0
     if diff.any():
         gap = (second[diff] - best[diff]) / np.maximum(second[diff], 1e-30)
-        assert gap.max() < ASSIGN_GAP, f"{what}: disagreement at relative gap {gap.max():.3e}"
+        gap_max = float(gap.max())
+    assert gap_max < ASSIGN_GAP, f"{what}: {int(diff.sum())} disagreement(s), relative gap up to {gap_max:.3e}"
+    assert agree >= ASSIGN_AGREE, f"{what}: agreement {agree:.6f} (gaps below {gap_max:.3e})"
     return agree, int(diff.sum())
 
 
