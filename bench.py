@@ -340,7 +340,7 @@ def run_gpu(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        info = cpu_oracle_sample(workload.get(WORKLOAD), head=0, iters=1, attn_rows=64)
+        info = cpu_oracle_sample(workload.get(WORKLOAD), head=0, iters=2, attn_rows=256)
         cpu = {"value": info["full_flops"] / info["est_seconds"] / 1e12, "unit": "TFLOPS", "cores": 1,
                "kind": "oracle", "sample": info["sample"],
                "est_ms_per_call": info["est_seconds"] * 1e3, "sample_seconds": info["sample_seconds"]}
