@@ -63,6 +63,7 @@ _SIGS = {
     "svoo_cluster_workspace_size": (_SZ, [_SP, _I, _I]),
     "svoo_cluster": (_I, [_SP, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _P]),
     "svoo_cluster_step": (_I, [_SP, _P, _I, _P, _P, _P, _P, _P, _I, _P, _SZ, _P, _P]),
+    "svoo_cluster_step_static": (_I, [_SP, _P, _I, _P, _P, _P, _P, _P, _I, _P, _P]),
     "svoo_mask_workspace_size": (_SZ, [_SP, _I, _I]),
     "svoo_build_mask": (_I, [_SP, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _PP, _P, _SZ,
                              _P, _P]),
@@ -260,6 +261,21 @@ def cluster_step(x, cent, sizes, assign, metric_cent=None, metric_sizes=None, n_
                                     _ptr(assign), _ptr(metric_cent), _ptr(metric_sizes), mC,
                                     _ptr(workspace), workspace.numel(), _ptr(err), _stream(stream)),
            "svoo_cluster_step")
+    return err
+
+
+def cluster_step_static(x, cent, sizes, assign, metric_cent=None, metric_sizes=None, n_text=0,
+                        dev_err=None, stream=None):
+    """cluster_step with the library's fixed device scratch instead of a
+    workspace (for callers that may not allocate device memory)."""
+    _need_cuda(x, cent, sizes, assign, metric_cent, metric_sizes)
+    sh = make_shape(x, n_text)
+    C = cent.shape[-2]
+    mC = metric_cent.shape[-2] if metric_cent is not None else 0
+    err = _err_buf(dev_err, x.device)
+    _check(load().svoo_cluster_step_static(ctypes.byref(sh), _ptr(x), C, _ptr(cent), _ptr(sizes),
+                                           _ptr(assign), _ptr(metric_cent), _ptr(metric_sizes), mC,
+                                           _ptr(err), _stream(stream)), "svoo_cluster_step_static")
     return err
 
 

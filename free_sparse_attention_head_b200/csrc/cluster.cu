@@ -545,3 +545,70 @@ extern "C" svoo_status svoo_cluster(const svoo_shape* shape, const void* q, cons
   }
   return SVOO_OK;
 }
+
+// ---------------------------------------------------------------- allocation-free variant
+//
+// svoo_cluster_step_static: the same half-step as svoo_cluster_step, with its
+// scratch in a fixed device array compiled into this library instead of a
+// caller-provided workspace. It is for callers that may not allocate device
+// memory themselves: code running inside a host framework that owns every
+// device allocation through its own pool and budget, or a latency-critical
+// loop whose policy forbids any allocation after start-up. The caller still
+// passes the inputs and outputs.
+//
+// The array costs kStaticScratchBytes on every GPU that loads this library,
+// until the process exits. Its device address is looked up once per device on
+// the first call made with that device current (so make the first call on each
+// device before any stream capture begins). Every call reuses the same array:
+// each call clears the accumulators it needs before using them, and calls whose
+// work overlaps on the GPU (for example on two streams) race on it.
+#include <mutex>
+
+namespace svoo {
+
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(16) << 20;
+static __device__ __align__(256) unsigned char g_step_scratch[kStaticScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 128;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_step_scratch for the current device (host code must not
+// use the symbol itself as a pointer: on the host it is only a stand-in).
+void* scratch_address(int* dev_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  *dev_out = dev;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_step_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    g_scratch_addr[dev] = p;
+  }
+  return g_scratch_addr[dev];
+}
+}  // namespace
+}  // namespace svoo
+
+extern "C" svoo_status svoo_cluster_step_static(const svoo_shape* shape, const void* x, int C,
+                                                float* cent, int32_t* sizes, int32_t* assign,
+                                                const float* metric_cent,
+                                                const int32_t* metric_sizes, int metric_C,
+                                                int32_t* dev_err, void* stream) {
+  if (!shape_ok(shape) || !x || !cent || !sizes || !assign) return SVOO_ERR_INVALID_ARG;
+  if (!cluster_counts_ok(C)) return SVOO_ERR_INVALID_ARG;
+  if (metric_cent && (!metric_sizes || !cluster_counts_ok(metric_C))) return SVOO_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return SVOO_ERR_INVALID_ARG;
+  const int BH = bh_of(shape);
+  const int Cmax = C > metric_C ? C : metric_C;
+  if (carve_step(nullptr, BH, shape->d, Cmax, nullptr) > kStaticScratchBytes)
+    return SVOO_ERR_WORKSPACE;  // shape needs more than the fixed scratch holds
+  int dev = 0;
+  void* base = scratch_address(&dev);
+  if (!base) return SVOO_ERR_CUDA;
+  StepWs w;
+  carve_step(base, BH, shape->d, Cmax, &w);
+  return run_step(shape, x, C, cent, sizes, assign, metric_cent, metric_sizes, metric_C, w, dev_err,
+                  static_cast<cudaStream_t>(stream), C);
+}

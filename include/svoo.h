@@ -138,6 +138,24 @@ svoo_status svoo_cluster_step(const svoo_shape *shape, const void *x, int C, flo
                               const int32_t *metric_sizes, int metric_C, void *workspace,
                               size_t workspace_bytes, int32_t *dev_err, void *stream);
 
+/* Allocation-free variant of svoo_cluster_step. The paper pages have no
+ * counterpart: it exists for callers that may not allocate device memory
+ * themselves (code inside a host framework that owns all device memory through
+ * its own pool, or a latency-critical loop that forbids allocation after
+ * start-up). Arguments as svoo_cluster_step minus the workspace; the scratch
+ * is a fixed array of SVOO_STATIC_SCRATCH_BYTES compiled into the library,
+ * held on every GPU that loads it until the process exits. Shapes whose
+ * scratch would exceed it return SVOO_ERR_WORKSPACE and enqueue nothing (16 MiB
+ * covers, e.g., B*H = 12, d = 128, 128 clusters). The first call on a device
+ * looks up the array's device address (make it before any stream capture).
+ * All calls share the array and each clears the accumulators it uses; calls
+ * that overlap on the GPU (e.g. on two streams) race. */
+#define SVOO_STATIC_SCRATCH_BYTES (16u << 20)
+svoo_status svoo_cluster_step_static(const svoo_shape *shape, const void *x, int C, float *cent,
+                                     int32_t *sizes, int32_t *assign, const float *metric_cent,
+                                     const int32_t *metric_sizes, int metric_C, int32_t *dev_err,
+                                     void *stream);
+
 /* ------------------------------------------------------------------ mask
  * Bytes of device workspace svoo_build_mask needs. */
 size_t svoo_mask_workspace_size(const svoo_shape *shape, int n_qc, int n_kc);

@@ -1,0 +1,85 @@
+"""svoo_cluster_step_static: the clustering half-step for callers that may not
+allocate device memory (a host framework that owns every device allocation
+through its own pool, or a loop that forbids allocation after start-up). Its
+scratch is a fixed array inside the library instead of a caller workspace.
+
+The test calls it through the C ABI twice in a row (a query step in feature
+space, then a key step under the query clusters' metric, so the second call
+runs on scratch the first one left behind) and checks each result against the
+workspace-based svoo_cluster_step on the same inputs. It also checks that a
+shape needing more than the fixed scratch is refused before any launch.
+This file sorts last so that a run stopping at its first failure has already
+run every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import workload
+import free_sparse_attention_head_b200 as svoo
+from free_sparse_attention_head_b200 import build as svoo_build
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev_bf16(a, B, H):
+    BH, N, d = a.shape
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16).view(B, H, N, d)
+
+
+def _token_start(x, C):
+    """Centroid j = token floor(j n / C), widened to fp32 (the library's cold start)."""
+    BH, n, d = x.shape
+    idx = [j * n // C for j in range(C)]
+    f = (x[:, idx, :].astype(np.uint32) << 16).view(np.float32)
+    return np.ascontiguousarray(f)
+
+
+def _step_both(xd, cent0, metric=None):
+    """Runs the workspace entry point and the static one on the same inputs."""
+    outs = []
+    for fn in (svoo.cluster_step, svoo.cluster_step_static):
+        BH, C, _ = cent0.shape
+        nv = xd.shape[2]
+        cent = torch.from_numpy(cent0.copy()).cuda()
+        sizes = torch.zeros(BH, C, dtype=torch.int32, device="cuda")
+        assign = torch.full((BH, nv), -1, dtype=torch.int32, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        mc, ms = (None, None) if metric is None else (metric[0], metric[1])
+        fn(xd, cent, sizes, assign, metric_cent=mc, metric_sizes=ms, dev_err=err)
+        torch.cuda.synchronize()
+        svoo.check_device_errors(err)
+        outs.append((assign, cent, sizes))
+    return outs
+
+
+def test_static_scratch_step_matches_workspace_step():
+    svoo_build.build()
+    svoo.load()
+    w = workload.get("wan2.1-1.3b")
+    import dataclasses
+    w = dataclasses.replace(w, H=2)
+    q, k, _ = workload.make_qkv(w)
+    qd, kd = _dev_bf16(q, w.B, w.H), _dev_bf16(k, w.B, w.H)
+    # call 1: query step, feature space
+    (a_ws, c_ws, s_ws), (a_st, c_st, s_st) = _step_both(qd, _token_start(q, w.n_qc))
+    assert torch.equal(a_ws, a_st)
+    assert torch.equal(s_ws, s_st)
+    assert torch.equal(c_ws.view(torch.int32), c_st.view(torch.int32))
+    assert int(s_st.sum()) == w.B * w.H * w.n_video
+    # call 2 (scratch still holds call 1's contents): key step under the query metric
+    (b_ws, d_ws, t_ws), (b_st, d_st, t_st) = _step_both(kd, _token_start(k, w.n_kc), metric=(c_st, s_st))
+    assert torch.equal(b_ws, b_st)
+    assert torch.equal(t_ws, t_st)
+    assert torch.equal(d_ws.view(torch.int32), d_st.view(torch.int32))
+
+
+def test_static_scratch_rejects_oversized_shape():
+    lib = svoo.load()
+    sh = svoo.Shape(1, 40, 75600, 128, 0)  # needs ~29 MB of scratch > 16 MiB
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: refused before any launch
+    st = lib.svoo_cluster_step_static(ctypes.byref(sh), fake, 256, fake, fake, fake, None, None, 0,
+                                      None, None)
+    assert st == 2 and lib.svoo_status_string(st) == b"workspace too small"
