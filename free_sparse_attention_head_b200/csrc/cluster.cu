@@ -24,9 +24,6 @@
 
 namespace svoo {
 
-constexpr int kAssignThreads = 128;  // one token row (= TMEM lane) per thread
-constexpr int kTileRows = 128;
-constexpr int kMaxCandidates = 8;
 
 // ---------------------------------------------------------------- init
 
@@ -41,138 +38,209 @@ __global__ void init_centroids_kernel(const uint16_t* __restrict__ x, int N, int
 
 // ---------------------------------------------------------------- metric
 
-// M[h] = sum_b n_b c_b c_b^T / sum_b n_b in fp64. grid (d/8, BH), block d
-// threads; thread j owns column j of rows i0..i0+7.
-__global__ void metric_m_kernel(const float* __restrict__ cent, const int32_t* __restrict__ sizes,
-                                int C, int d, double* __restrict__ M) {
-  extern __shared__ double sm_m[];  // [32][d] centroid chunk, then [32] sizes
-  double* cch = sm_m;
-  double* nch = sm_m + 32 * d;
-  const int h = blockIdx.y, i0 = blockIdx.x * 8, j = threadIdx.x;
-  double acc[8];
-#pragma unroll
-  for (int r = 0; r < 8; ++r) acc[r] = 0.0;
+// M[h] = sum_b n_b c_b c_b^T / sum_b n_b in fp64. grid (T*(T+1)/2, BH) with
+// T = d/16 output tiles per side (upper triangle only; each tile is written
+// to both (i, j) and (j, i), so M is exactly symmetric), block 256 = 16 x 16,
+// one output per thread; clusters staged 64 at a time.
+constexpr int kMetricChunk = 64;
+
+__global__ void __launch_bounds__(256)
+    metric_m_kernel(const float* __restrict__ cent, const int32_t* __restrict__ sizes, int C, int d,
+                    double* __restrict__ M) {
+  __shared__ double ci[kMetricChunk][17];
+  __shared__ double cj[kMetricChunk][17];
+  const int h = blockIdx.y, T = d / 16;
+  int t = blockIdx.x, ti = 0;
+  while (t >= T - ti) {  // upper-triangle tile index -> (ti, tj), ti <= tj
+    t -= T - ti;
+    ++ti;
+  }
+  const int tj = ti + t;
+  const int a = threadIdx.x >> 4, b = threadIdx.x & 15;
+  const int i0 = ti * 16, j0 = tj * 16;
+  double acc = 0.0;
   long long total = 0;
-  for (int b0 = 0; b0 < C; b0 += 32) {
-    int nb = min(32, C - b0);
+  for (int b0 = 0; b0 < C; b0 += kMetricChunk) {
+    const int nb = min(kMetricChunk, C - b0);
     __syncthreads();
-    for (int e = threadIdx.x; e < nb * d; e += blockDim.x)
-      cch[e] = static_cast<double>(cent[(static_cast<size_t>(h) * C + b0) * d + e]);
-    if (threadIdx.x < nb) nch[threadIdx.x] = static_cast<double>(sizes[h * C + b0 + threadIdx.x]);
-    __syncthreads();
-    for (int bb = 0; bb < nb; ++bb) {
-      double n = nch[bb];
-      total += static_cast<long long>(n);
-      if (n == 0.0) continue;
-      double cj = n * cch[bb * d + j];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) acc[r] = fma(cch[bb * d + i0 + r], cj, acc[r]);
+    for (int e = threadIdx.x; e < nb * 16; e += blockDim.x) {
+      const int bb = e >> 4, c = e & 15;
+      const float* cb = cent + (static_cast<size_t>(h) * C + b0 + bb) * d;
+      const double n = static_cast<double>(sizes[h * C + b0 + bb]);
+      ci[bb][c] = n * static_cast<double>(cb[i0 + c]);
+      cj[bb][c] = static_cast<double>(cb[j0 + c]);
     }
+    __syncthreads();
+    for (int bb = 0; bb < nb; ++bb) acc = fma(ci[bb][a], cj[bb][b], acc);
   }
-#pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    double v = total > 0 ? acc[r] / static_cast<double>(total) : (i0 + r == j ? 1.0 : 0.0);
-    M[(static_cast<size_t>(h) * d + i0 + r) * d + j] = v;
-  }
+  for (int bb = 0; bb < C; ++bb) total += sizes[h * C + bb];
+  const double v = total > 0 ? acc / static_cast<double>(total) : ((i0 + a) == (j0 + b) ? 1.0 : 0.0);
+  double* Mh = M + static_cast<size_t>(h) * d * d;
+  Mh[static_cast<size_t>(i0 + a) * d + j0 + b] = v;
+  if (ti != tj) Mh[static_cast<size_t>(j0 + b) * d + i0 + a] = v;
 }
 
-// nu_j = M mu_j (M symmetric, read by columns), kappa_j = mu_j . nu_j in fp64;
-// also bf16(nu_j) for the scoring MMA, fp32 kappa and |nu_j| for its error
-// bound. Clusters j in [C, Cpad) are padding (nu = 0, kappa = +inf).
-// grid (Cpad/8, BH), block d threads; M == nullptr means identity.
-__global__ void metric_nu_kernel(const double* __restrict__ M, const float* __restrict__ cent, int C,
-                                 int Cpad, int d, double* __restrict__ nu64,
-                                 uint16_t* __restrict__ nu_bf16, double* __restrict__ kappa64,
-                                 float* __restrict__ kappa32, float* __restrict__ nunorm) {
-  extern __shared__ double sm_nu[];  // [8][d] mu rows, [8][4][2] reduction scratch
-  double* mu = sm_nu;
-  double* red = sm_nu + 8 * d;
-  const int h = blockIdx.y, j0 = blockIdx.x * 8, i = threadIdx.x;
-  for (int e = threadIdx.x; e < 8 * d; e += blockDim.x) {
-    int r = e / d, c = e % d;
-    mu[e] = (j0 + r < C) ? static_cast<double>(cent[(static_cast<size_t>(h) * C + j0 + r) * d + c]) : 0.0;
+// nu_j = M mu_j, kappa_j = mu_j . nu_j (fp64), bf16(nu_j), fp32 kappa and |nu_j|;
+// clusters j in [C, Cpad) are padding (nu = 0, kappa = +inf). grid (Cpad/32, BH),
+// block 256: warp w owns clusters j0 + 4w .. +3, lane owns dimensions 4 lane .. +3
+// (d = 128; for d = 64 lanes 16..31 idle). M == nullptr means identity.
+__global__ void __launch_bounds__(256)
+    metric_nu_kernel(const double* __restrict__ M, const float* __restrict__ cent, int C, int Cpad,
+                     int d, double* __restrict__ nu64, uint16_t* __restrict__ nu_bf16,
+                     double* __restrict__ kappa64, float* __restrict__ kappa32,
+                     float* __restrict__ nunorm) {
+  __shared__ float mu[32][129];      // this block's 32 clusters, all dimensions (exact fp32)
+  __shared__ double mch[16][128];    // 16 rows of M
+  const int h = blockIdx.y, j0 = blockIdx.x * 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < 32 * d; e += blockDim.x) {
+    const int r = e / d, c = e % d;
+    mu[r][c] = (j0 + r < C) ? cent[(static_cast<size_t>(h) * C + j0 + r) * d + c] : 0.f;
   }
-  __syncthreads();
-  double acc[8];
+  const bool live = 4 * lane < d;
+  double acc[4][4];  // [cluster][dimension]
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.0;
   if (M) {
-#pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r] = 0.0;
     const double* Mh = M + static_cast<size_t>(h) * d * d;
-    for (int l = 0; l < d; ++l) {
-      double m = Mh[static_cast<size_t>(l) * d + i];
+    for (int l0 = 0; l0 < d; l0 += 16) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < 16 * d; e += blockDim.x) mch[e / d][e % d] = Mh[static_cast<size_t>(l0) * d + e];
+      __syncthreads();
+      if (live) {
+        for (int l = 0; l < 16; ++l) {
+          // M symmetric: nu_j[i] = sum_l M[l][i] mu_j[l]
+          const double2 m01 = *reinterpret_cast<const double2*>(&mch[l][4 * lane]);
+          const double2 m23 = *reinterpret_cast<const double2*>(&mch[l][4 * lane + 2]);
+          const double mv[4] = {m01.x, m01.y, m23.x, m23.y};
 #pragma unroll
-      for (int r = 0; r < 8; ++r) acc[r] = fma(m, mu[r * d + l], acc[r]);
+          for (int u = 0; u < 4; ++u) {
+            const double m_u = static_cast<double>(mu[4 * warp + u][l0 + l]);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[u][v] = fma(mv[v], m_u, acc[u][v]);
+          }
+        }
+      }
     }
   } else {
+    __syncthreads();
+    if (live)
 #pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r] = mu[r * d + i];
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = static_cast<double>(mu[4 * warp + u][4 * lane + v]);
   }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    int j = j0 + r;
-    size_t o = (static_cast<size_t>(h) * Cpad + j) * d + i;
-    if (j < C) nu64[(static_cast<size_t>(h) * C + j) * d + i] = acc[r];
-    __nv_bfloat16 b = __float2bfloat16_rn(j < C ? static_cast<float>(acc[r]) : 0.f);
-    nu_bf16[o] = *reinterpret_cast<uint16_t*>(&b);
-    double k1 = mu[r * d + i] * acc[r];
-    double k2 = acc[r] * acc[r];
-    for (int s = 16; s > 0; s >>= 1) {
-      k1 += __shfl_xor_sync(0xffffffffu, k1, s);
-      k2 += __shfl_xor_sync(0xffffffffu, k2, s);
+  for (int u = 0; u < 4; ++u) {
+    const int j = j0 + 4 * warp + u;
+    double k1 = 0.0, k2 = 0.0;
+    if (live) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int i = 4 * lane + v;
+        k1 = fma(static_cast<double>(mu[4 * warp + u][i]), acc[u][v], k1);
+        k2 = fma(acc[u][v], acc[u][v], k2);
+        if (j < C) nu64[(static_cast<size_t>(h) * C + j) * d + i] = acc[u][v];
+        __nv_bfloat16 bv = __float2bfloat16_rn(j < C ? static_cast<float>(acc[u][v]) : 0.f);
+        nu_bf16[(static_cast<size_t>(h) * Cpad + j) * d + i] = *reinterpret_cast<uint16_t*>(&bv);
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      k1 += __shfl_xor_sync(0xffffffffu, k1, o);
+      k2 += __shfl_xor_sync(0xffffffffu, k2, o);
     }
     if (lane == 0) {
-      red[(r * 4 + warp) * 2 + 0] = k1;
-      red[(r * 4 + warp) * 2 + 1] = k2;
+      kappa64[h * Cpad + j] = j < C ? k1 : INFINITY;
+      kappa32[h * Cpad + j] = j < C ? static_cast<float>(k1) : INFINITY;
+      nunorm[h * Cpad + j] = j < C ? static_cast<float>(sqrt(k2)) : 0.f;
     }
-  }
-  __syncthreads();
-  if (threadIdx.x < 8) {
-    int r = threadIdx.x, j = j0 + r;
-    double k1 = 0.0, k2 = 0.0;
-    for (int w = 0; w < nwarp; ++w) {
-      k1 += red[(r * 4 + w) * 2 + 0];
-      k2 += red[(r * 4 + w) * 2 + 1];
-    }
-    kappa64[h * Cpad + j] = j < C ? k1 : INFINITY;
-    kappa32[h * Cpad + j] = j < C ? static_cast<float>(k1) : INFINITY;
-    nunorm[h * Cpad + j] = j < C ? static_cast<float>(sqrt(k2)) : 0.f;
   }
 }
 
 // ---------------------------------------------------------------- assign + update
+//
+// One CTA (256 threads) walks `tiles_per_cta` tiles of 128 tokens of one head.
+// Per tile: TMA load of X (128B-swizzled K-major), one tcgen05 MMA chain
+// X . bf16(nu)^T into TMEM (128 lanes x Cpad fp32 columns). Thread (r, h)
+// (warps w and w + 4 share TMEM lanes 32(w % 4).., h = w / 4) owns half h of
+// row r's scores s_j = kappa_j - 2 x.nu_j. Pass 1 finds the half's minimum;
+// with the row minimum m and the MMA error bound E, pass 2 lists the columns
+// with s_j <= m + 2E (they contain the exact argmin). A row with a single
+// candidate takes it; otherwise one warp re-scores its candidates in fp64
+// (kappa_j - 2 x.nu_j, dimensions split over the lanes) and the minimum wins,
+// ties to the smaller j. The tile's tokens are then grouped by label (counting
+// sort in shared memory) and each label run of each (4-dimension group, slice)
+// is summed in fp64 and added to the head's sums with one atomic per run.
+
+constexpr int kAssignThreads = 256;
+constexpr int kTileRows = 128;
+constexpr int kSlots = 8;  // candidate slots per half-row; more -> full re-score
 
 struct AssignSmem {
   int abort;
   uint32_t tmem_base;
   uint64_t tma_bar;
   uint64_t mma_bar;
+  float max_nrm;
+  float max_kap;
+  int namb;
+  float xn2[2][kTileRows];
+  float mh[2][kTileRows];
+  int kc[2][kTileRows];                 // candidates per half (kSlots + 1 = overflow)
+  int16_t slot[kTileRows][2][kSlots];
   int lab[kTileRows];
-  uint32_t keys[kTileRows];
+  int pos[kTileRows];
+  int16_t amb[kTileRows];
+  int16_t sorted_row[kTileRows];
+  int16_t sorted_lab[kTileRows];
+  int lstart[256];
+  int wsum[8];
+  float red[8];
 };
+constexpr int kAssignHeader = 12288;  // AssignSmem + per-CTA counts, keeps the X tile 1024-aligned
+static_assert(sizeof(AssignSmem) + 256 * sizeof(int) <= kAssignHeader, "header overflow");
 
-constexpr int kAssignHeader = 2048;  // AssignSmem, padded so the X tile stays 1024-aligned
-static_assert(sizeof(AssignSmem) <= kAssignHeader, "header overflow");
+// bf16 pair (columns c, c+1, c even) of row `row` in a 128-row swizzled X tile
+__device__ __forceinline__ uint32_t x_pair(const uint8_t* xs, int row, int c) {
+  return *reinterpret_cast<const uint32_t*>(xs + sw128_offset(row, c, kTileRows));
+}
 
-// grid (ceil(ntiles / tiles_per_cta), BH), block 128.
-// Dynamic smem: [AssignSmem, 2 KB][X tile 128 x d bf16][nu Cpad x d bf16][kappa][nunorm]
-__global__ void __launch_bounds__(kAssignThreads)
+// fp64 score kappa_j - 2 x_row . nu_j, computed by the whole warp (lane = 2 or 4 dims)
+__device__ __forceinline__ double warp_score(const uint8_t* xs, int row, const double* nj, double kap,
+                                             int d, int lane) {
+  double part = 0.0;
+  for (int c = lane * 2; c < d; c += 64) {
+    const uint32_t xp = x_pair(xs, row, c);
+    const double2 n2 = *reinterpret_cast<const double2*>(nj + c);
+    part = fma(static_cast<double>(__uint_as_float(xp << 16)), n2.x, part);
+    part = fma(static_cast<double>(__uint_as_float(xp & 0xffff0000u)), n2.y, part);
+  }
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  return kap - 2.0 * part;
+}
+
+// grid (ceil(ntiles / tiles_per_cta), BH), block 256.
+// Dynamic smem: [AssignSmem + counts, 12 KB][X tile 128 x d bf16][nu Cpad x d bf16][kappa][nunorm]
+__global__ void __launch_bounds__(kAssignThreads, 2)
     assign_update_kernel(const __grid_constant__ CUtensorMap xmap, int N, int nv, int d, int C,
                          int Cpad, int tmem_cols, int tiles_per_cta,
                          const uint16_t* __restrict__ nu_bf16, const double* __restrict__ nu64,
                          const double* __restrict__ kappa64, const float* __restrict__ kappa_g,
-                         const float* __restrict__ nunorm_g,
-                         int32_t* __restrict__ assign, double* __restrict__ sums,
-                         int32_t* __restrict__ counts, int* __restrict__ err) {
+                         const float* __restrict__ nunorm_g, int32_t* __restrict__ assign,
+                         double* __restrict__ sums, int32_t* __restrict__ counts,
+                         int* __restrict__ err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   AssignSmem* S = reinterpret_cast<AssignSmem*>(base);
+  int* cnt = reinterpret_cast<int*>(base + sizeof(AssignSmem));
   uint8_t* xs = base + kAssignHeader;
   uint8_t* nus = xs + kTileRows * d * 2;
   float* kap = reinterpret_cast<float*>(nus + static_cast<size_t>(Cpad) * d * 2);
   float* nrm = kap + Cpad;
 
-  const int h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+  const int h = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ntiles = (nv + kTileRows - 1) / kTileRows;
   const int t_begin = blockIdx.x * tiles_per_cta;
   const int t_end = min(ntiles, t_begin + tiles_per_cta);
@@ -190,7 +258,7 @@ __global__ void __launch_bounds__(kAssignThreads)
     tmem_alloc(smem_u32(&S->tmem_base), tmem_cols);
     tmem_relinquish();
   }
-  // nu (bf16) into the 128B-swizzled K-major layout the MMA expects.
+  // nu (bf16) into the 128B-swizzled K-major layout the MMA expects; kappa, |nu|
   {
     const int chunks = d / 8;
     const uint4* src = reinterpret_cast<const uint4*>(nu_bf16 + static_cast<size_t>(h) * Cpad * d);
@@ -198,9 +266,32 @@ __global__ void __launch_bounds__(kAssignThreads)
       int j = e / chunks, c = e % chunks;
       *reinterpret_cast<uint4*>(nus + sw128_offset(j, c * 8, Cpad)) = src[e];
     }
+    float mn = 0.f, mk = 0.f;
     for (int j = tid; j < Cpad; j += blockDim.x) {
       kap[j] = kappa_g[h * Cpad + j];
       nrm[j] = nunorm_g[h * Cpad + j];
+      cnt[j] = 0;
+      mn = fmaxf(mn, nrm[j]);
+      if (j < C) mk = fmaxf(mk, fabsf(kap[j]));
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fmaxf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
+    }
+    if (lane == 0) S->red[warp] = mn;
+    __syncthreads();
+    if (tid == 0) {
+      float a = 0.f;
+      for (int w = 0; w < 8; ++w) a = fmaxf(a, S->red[w]);
+      S->max_nrm = a;
+    }
+    __syncthreads();
+    if (lane == 0) S->red[warp] = mk;
+    __syncthreads();
+    if (tid == 0) {
+      float a = 0.f;
+      for (int w = 0; w < 8; ++w) a = fmaxf(a, S->red[w]);
+      S->max_kap = a;
     }
   }
   fence_proxy_async_smem();
@@ -215,19 +306,25 @@ __global__ void __launch_bounds__(kAssignThreads)
   const double* nu_h = nu64 + static_cast<size_t>(h) * C * d;
   const double* kap64 = kappa64 + static_cast<size_t>(h) * Cpad;
   const size_t xrow0 = static_cast<size_t>(h) * N;
+  const int r = ((warp & 3) << 5) | lane;  // token row == TMEM lane
+  const int half = warp >> 2;
+  const int ncol = Cpad / 2;               // columns of this thread's half
+  const int col0 = half * ncol;
+  const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + col0;
+  const float max_nrm = S->max_nrm, max_kap = S->max_kap;
 
   int it = 0;
-  int tma_pending = -1;  // parity of a TMA phase issued but not yet seen complete
+  int tma_pending = -1;
   for (int t = t_begin; t < t_end; ++t, ++it) {
     const uint32_t par = it & 1;
     if (tid == 0) {
       tma_pending = static_cast<int>(par);
+      S->namb = 0;
       mbar_arrive_expect_tx(smem_u32(&S->tma_bar), kTileRows * d * 2);
       for (int s = 0; s < d / 64; ++s)
         tma_load_2d(&xmap, xs_u32 + s * kTileRows * 128, smem_u32(&S->tma_bar), s * 64,
                     static_cast<int>(xrow0 + static_cast<size_t>(t) * kTileRows));
-      bool ok = mbar_wait(smem_u32(&S->tma_bar), par, abort);
-      if (ok) {
+      if (mbar_wait(smem_u32(&S->tma_bar), par, abort)) {
         tma_pending = -1;
         tc_fence_after();
         for (int kk = 0; kk < d / 16; ++kk) {
@@ -239,147 +336,198 @@ __global__ void __launch_bounds__(kAssignThreads)
         umma_commit(smem_u32(&S->mma_bar));
       }
     }
-    // warp-uniform verdict: the tcgen05.ld below is warp-collective
-    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&S->mma_bar), par, abort))) break;
+    if (tid < Cpad) S->lstart[tid] = 0;
+    // a CTA-uniform verdict keeps every barrier below matched
+    if (__syncthreads_or(mbar_wait(smem_u32(&S->mma_bar), par, abort) ? 0 : 1)) break;
     tc_fence_after();
-
-    // ---- per-token argmin with error bound and fp32 recheck
-    const int r = tid;
     const int tok = t * kTileRows + r;
     const bool valid = tok < nv;
-    const uint8_t* xrow = xs;  // element (r, c) at sw128_offset(r, c, 128)
-    float xn2 = 0.f;
-    for (int c = 0; c < d; ++c) {
-      float v = bf16_to_f32(*reinterpret_cast<const uint16_t*>(xrow + sw128_offset(r, c, kTileRows)));
-      xn2 = fmaf(v, v, xn2);
-    }
-    // |x.nu - acc| <= 2^-8 |x||nu| covers bf16 rounding of nu (2^-9) plus the
-    // fp32 accumulation; the score kappa - 2 x.nu therefore errs by at most
-    // 2^-7 |x||nu|. Use 2^-6 for margin.
-    const float eps_x = ldexpf(sqrtf(xn2), -6);
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float U = INFINITY;
-    for (int q = 0; q < Cpad / 32; ++q) {
-      uint32_t v[32];
-      tmem_ld32(lane_addr + q * 32, v);
-      tmem_wait_ld();
+    // ---- partial |x|^2 over this half of the dimensions; pass 1: the half's minimum
+    {
+      float acc = 0.f;
+      const int dh = d / 2;
+      for (int c = half * dh; c < (half + 1) * dh; c += 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xs + sw128_offset(r, c, kTileRows));
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        int j = q * 32 + c;
-        float s = kap[j] - 2.f * __uint_as_float(v[c]);
-        U = fminf(U, s + eps_x * nrm[j]);
-      }
-    }
-    int cand[kMaxCandidates];
-    int ncand = 0;
-    bool overflow = false;
-    for (int q = 0; q < Cpad / 32; ++q) {
-      uint32_t v[32];
-      tmem_ld32(lane_addr + q * 32, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        int j = q * 32 + c;
-        float s = kap[j] - 2.f * __uint_as_float(v[c]);
-        if (s - eps_x * nrm[j] <= U) {
-          if (ncand < kMaxCandidates) cand[ncand] = j;
-          else overflow = true;
-          ++ncand;
+        for (int q = 0; q < 4; ++q) {
+          const float lo = __uint_as_float(w4[q] << 16), hi = __uint_as_float(w4[q] & 0xffff0000u);
+          acc = fmaf(lo, lo, fmaf(hi, hi, acc));
         }
       }
+      S->xn2[half][r] = acc;
+      float m = INFINITY;
+      for (int q = 0; q < ncol / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + q * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 k4 = *reinterpret_cast<const float4*>(kap + col0 + q * 32 + c);
+          m = fminf(m, fminf(fminf(fmaf(-2.f, __uint_as_float(v[c]), k4.x), fmaf(-2.f, __uint_as_float(v[c + 1]), k4.y)),
+                             fminf(fmaf(-2.f, __uint_as_float(v[c + 2]), k4.z), fmaf(-2.f, __uint_as_float(v[c + 3]), k4.w))));
+        }
+      }
+      S->mh[half][r] = m;
+    }
+    __syncthreads();
+    // ---- pass 2: every column within 2E of the row minimum is a candidate.
+    // |score error| <= 2 (2^-9 + d 2^-23) |x| |nu_j| (bf16 nu, fp32 accumulation)
+    // plus fp32 rounding of kappa and of the score; 2^-6 |x| max|nu| (+ a
+    // relative slack) covers it with margin. Both halves compute the same thr.
+    {
+      const float m = fminf(S->mh[0][r], S->mh[1][r]);
+      const float xn = sqrtf(S->xn2[0][r] + S->xn2[1][r]);
+      const float E = ldexpf(xn * max_nrm, -6) + ldexpf(max_kap + 2.f * xn * max_nrm, -20);
+      const float thr = m + 2.f * E;
+      int k = 0;
+      for (int q = 0; q < ncol / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + q * 32, v);
+        tmem_wait_ld();
+        uint32_t bits = 0;  // candidates of this 32-column chunk (padding has kappa = +inf)
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+          const float4 k4 = *reinterpret_cast<const float4*>(kap + col0 + q * 32 + c);
+          bits |= (fmaf(-2.f, __uint_as_float(v[c]), k4.x) <= thr ? 1u : 0u) << c;
+          bits |= (fmaf(-2.f, __uint_as_float(v[c + 1]), k4.y) <= thr ? 1u : 0u) << (c + 1);
+          bits |= (fmaf(-2.f, __uint_as_float(v[c + 2]), k4.z) <= thr ? 1u : 0u) << (c + 2);
+          bits |= (fmaf(-2.f, __uint_as_float(v[c + 3]), k4.w) <= thr ? 1u : 0u) << (c + 3);
+        }
+        while (bits) {
+          const int c = __ffs(bits) - 1;
+          bits &= bits - 1;
+          if (k < kSlots) S->slot[r][half][k] = static_cast<int16_t>(col0 + q * 32 + c);
+          ++k;
+        }
+      }
+      S->kc[half][r] = k;
     }
     tc_fence_before();
-    // Decision: a single candidate is the argmin; otherwise the candidates
-    // are re-scored exactly as the definition reads, kappa_j - 2 x.nu_j in
-    // fp64 (nu, kappa from the fp64 metric), ties to the smaller j.
-    int best_j = 0;
-    auto exact_score = [&](int j) -> double {
-      const double* nj = nu_h + static_cast<size_t>(j) * d;
-      double dot = 0.0;
-      for (int c = 0; c < d; ++c) {
-        float xv = bf16_to_f32(*reinterpret_cast<const uint16_t*>(xrow + sw128_offset(r, c, kTileRows)));
-        dot = fma(static_cast<double>(xv), __ldg(nj + c), dot);
-      }
-      return kap64[j] - 2.0 * dot;
-    };
-    if (valid) {
-      if (ncand == 1) {
-        best_j = cand[0];
-      } else {
-        double best = INFINITY;
-        const int n_eval = overflow ? C : ncand;
-        for (int k = 0; k < n_eval; ++k) {
-          const int j = overflow ? k : cand[k < kMaxCandidates ? k : 0];
-          const double s = exact_score(j);
-          if (s < best) {  // candidates ascend in j: ties keep the smaller j
-            best = s;
-            best_j = j;
-          }
-        }
-      }
-      assign[static_cast<size_t>(h) * nv + tok] = best_j;
-    }
-    S->lab[r] = valid ? best_j : -1;
-    S->keys[r] = (static_cast<uint32_t>(valid ? best_j + 1 : 0) << 8) | static_cast<uint32_t>(r);
     __syncthreads();
-
-    // ---- bitonic sort of (label, row) keys, 128 entries, one per thread
-    for (int k = 2; k <= kTileRows; k <<= 1) {
-      for (int jj = k >> 1; jj > 0; jj >>= 1) {
-        int ixj = r ^ jj;
-        if (ixj > r) {
-          uint32_t a = S->keys[r], b = S->keys[ixj];
-          bool up = (r & k) == 0;
-          if ((a > b) == up) {
-            S->keys[r] = b;
-            S->keys[ixj] = a;
+    // ---- rows with one candidate take it; the others are queued for fp64 re-scoring
+    if (half == 0) {
+      const int k0 = S->kc[0][r], k1 = S->kc[1][r];
+      int L = -1;
+      if (valid) {
+        if (k0 + k1 == 1) {
+          L = k0 ? S->slot[r][0][0] : S->slot[r][1][0];
+        } else {
+          S->amb[atomicAdd(&S->namb, 1)] = static_cast<int16_t>(r);
+        }
+      }
+      S->lab[r] = L;
+    }
+    __syncthreads();
+    // ---- one warp per ambiguous row: candidates in ascending j, strict minimum
+    const int namb = S->namb;
+    for (int a = warp; a < namb; a += 8) {
+      const int rr = S->amb[a];
+      const int k0 = S->kc[0][rr], k1 = S->kc[1][rr];
+      double best = INFINITY;
+      int bj = 0;
+      if (k0 <= kSlots && k1 <= kSlots) {
+        for (int q = 0; q < k0 + k1; ++q) {
+          const int j = q < k0 ? S->slot[rr][0][q] : S->slot[rr][1][q - k0];
+          const double sc = warp_score(xs, rr, nu_h + static_cast<size_t>(j) * d, kap64[j], d, lane);
+          if (sc < best) {
+            best = sc;
+            bj = j;
           }
         }
-        __syncthreads();
+      } else {  // too many candidates for the slots: re-score every cluster
+        for (int j = 0; j < C; ++j) {
+          const double sc = warp_score(xs, rr, nu_h + static_cast<size_t>(j) * d, kap64[j], d, lane);
+          if (sc < best) {
+            best = sc;
+            bj = j;
+          }
+        }
       }
+      if (lane == 0) S->lab[rr] = bj;
     }
-    // ---- run sums (exact fp64) -> atomics; thread = dimension
-    if (r < d) {
+    __syncthreads();
+    // ---- labels out; counting sort of the tile's rows by label
+    if (half == 0 && valid) {
+      const int L = S->lab[r];
+      assign[static_cast<size_t>(h) * nv + tok] = L;
+      S->pos[r] = atomicAdd(&S->lstart[L], 1);
+    }
+    __syncthreads();
+    if (tid < Cpad) {  // exclusive scan of the label histogram (Cpad <= 256 threads)
+      const int c0 = S->lstart[tid];
+      cnt[tid] += c0;
+      int inc = c0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (lane == 31) S->wsum[warp] = inc;
+      S->lstart[tid] = inc - c0;
+    }
+    __syncthreads();
+    if (tid < Cpad) {
+      int add = 0;
+      for (int w = 0; w < warp; ++w) add += S->wsum[w];
+      S->lstart[tid] += add;
+    }
+    __syncthreads();
+    if (half == 0 && valid) {
+      const int L = S->lab[r];
+      const int p = S->lstart[L] + S->pos[r];
+      S->sorted_row[p] = static_cast<int16_t>(r);
+      S->sorted_lab[p] = static_cast<int16_t>(L);
+    }
+    __syncthreads();
+    // ---- run sums in fp64: thread = (4-dimension group, slice of the sorted rows)
+    {
+      const int nvalid = min(kTileRows, nv - t * kTileRows);
+      const int ngrp = d / 4;
+      const int slices = kAssignThreads / ngrp;
+      const int per = kTileRows / slices;
+      const int g = tid % ngrp, sl = tid / ngrp;
+      const int c4 = 4 * g;
       int cur = -1;
-      double acc = 0.0;
-      for (int p = 0; p < kTileRows; ++p) {
-        uint32_t key = S->keys[p];
-        int lbl = static_cast<int>(key >> 8) - 1;
-        if (lbl < 0) continue;
-        int row = key & 255;
-        if (lbl != cur) {
-          if (cur >= 0) atomicAdd(&sums[(static_cast<size_t>(h) * C + cur) * d + r], acc);
-          cur = lbl;
-          acc = 0.0;
+      double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+      auto flush = [&]() {
+        double* dst = sums + (static_cast<size_t>(h) * C + cur) * d + c4;
+        atomicAdd(dst, a0);
+        atomicAdd(dst + 1, a1);
+        atomicAdd(dst + 2, a2);
+        atomicAdd(dst + 3, a3);
+      };
+      const int pend = min(nvalid, (sl + 1) * per);
+      for (int p = sl * per; p < pend; ++p) {
+        const int L = S->sorted_lab[p];
+        if (L != cur) {
+          if (cur >= 0) flush();
+          cur = L;
+          a0 = a1 = a2 = a3 = 0.0;
         }
-        float v = bf16_to_f32(*reinterpret_cast<const uint16_t*>(xrow + sw128_offset(row, r, kTileRows)));
-        if (fabsf(v) < 5.9604644775390625e-08f) v = 0.f;  // 2^-24
-        acc += static_cast<double>(v);
+        const uint2 q2 = *reinterpret_cast<const uint2*>(xs + sw128_offset(S->sorted_row[p], c4, kTileRows));
+        float f0 = __uint_as_float(q2.x << 16), f1 = __uint_as_float(q2.x & 0xffff0000u);
+        float f2 = __uint_as_float(q2.y << 16), f3 = __uint_as_float(q2.y & 0xffff0000u);
+        // components below 2^-24 count as zero (exact, order-independent sums)
+        f0 = fabsf(f0) < 5.9604644775390625e-08f ? 0.f : f0;
+        f1 = fabsf(f1) < 5.9604644775390625e-08f ? 0.f : f1;
+        f2 = fabsf(f2) < 5.9604644775390625e-08f ? 0.f : f2;
+        f3 = fabsf(f3) < 5.9604644775390625e-08f ? 0.f : f3;
+        a0 += static_cast<double>(f0);
+        a1 += static_cast<double>(f1);
+        a2 += static_cast<double>(f2);
+        a3 += static_cast<double>(f3);
       }
-      if (cur >= 0) atomicAdd(&sums[(static_cast<size_t>(h) * C + cur) * d + r], acc);
-    }
-    if (r == (d < kTileRows ? d : 0)) {
-      // one thread counts the runs (d < 128: a thread outside the sum loop)
-      int cur = -1, len = 0;
-      for (int p = 0; p < kTileRows; ++p) {
-        int lbl = static_cast<int>(S->keys[p] >> 8) - 1;
-        if (lbl < 0) continue;
-        if (lbl != cur) {
-          if (cur >= 0) atomicAdd(&counts[h * C + cur], len);
-          cur = lbl;
-          len = 0;
-        }
-        ++len;
-      }
-      if (cur >= 0) atomicAdd(&counts[h * C + cur], len);
+      if (cur >= 0) flush();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
   }
+  __syncthreads();
+  for (int j = tid; j < C; j += blockDim.x)
+    if (cnt[j]) atomicAdd(&counts[h * C + j], cnt[j]);
   if (*abort && tid == 0) {
     report_error(err, kErrTimeoutCluster);
-    // never leave with a copy still writing into this CTA's shared memory
     if (tma_pending >= 0) {
       int dummy = 0;
       mbar_wait(smem_u32(&S->tma_bar), static_cast<uint32_t>(tma_pending), &dummy);
@@ -425,7 +573,7 @@ struct StepWs {
 
 size_t carve_step(void* ws, int BH, int d, int Cmax, StepWs* out) {
   Carver cv(ws);
-  int Cpad = pad32(Cmax);
+  int Cpad = pad64(Cmax);
   StepWs w;
   w.M = cv.take<double>(static_cast<size_t>(BH) * d * d);
   w.nu64 = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
@@ -456,7 +604,7 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
                      int metric_C, const StepWs& w, int32_t* dev_err, cudaStream_t st,
                      int zero_C) {
   const int BH = bh_of(sh), d = sh->d, N = sh->N, nv = nvideo_of(sh);
-  const int Cpad = pad32(C);
+  const int Cpad = pad64(C);
   // finalize_kernel re-zeroes what a step used, so only the first step of a
   // call clears the accumulators (for the largest cluster count of the call).
   if (zero_C > 0) {
@@ -465,16 +613,16 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
       return SVOO_ERR_CUDA;
   }
   if (metric_cent) {
-    metric_m_kernel<<<dim3(d / 8, BH), d, (32 * d + 32) * sizeof(double), st>>>(metric_cent, metric_sizes,
-                                                                                metric_C, d, w.M);
+    const int T = d / 16;
+    metric_m_kernel<<<dim3(T * (T + 1) / 2, BH), 256, 0, st>>>(metric_cent, metric_sizes, metric_C, d, w.M);
   }
-  metric_nu_kernel<<<dim3(Cpad / 8, BH), d, (8 * d + 64) * sizeof(double), st>>>(
-      metric_cent ? w.M : nullptr, cent, C, Cpad, d, w.nu64, w.nu_bf16, w.kappa64, w.kappa, w.nunorm);
+  metric_nu_kernel<<<dim3(Cpad / 32, BH), 256, 0, st>>>(metric_cent ? w.M : nullptr, cent, C, Cpad, d,
+                                                        w.nu64, w.nu_bf16, w.kappa64, w.kappa, w.nunorm);
   CUtensorMap xmap;
   if (encode_tiled_2d(&xmap, x, static_cast<uint64_t>(BH) * N, d, kTileRows, 64) != CUDA_SUCCESS)
     return SVOO_ERR_CUDA;
   const int ntiles = (nv + kTileRows - 1) / kTileRows;
-  const int tpc = ntiles >= 64 ? 8 : 1;
+  const int tpc = ntiles >= 128 ? 16 : (ntiles >= 16 ? 4 : 1);
   const size_t smem = assign_smem_bytes(d, Cpad);
   if (cudaFuncSetAttribute(assign_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)

@@ -32,9 +32,9 @@ inline int mask_words(const svoo_shape* s, int n_kc) { return (groups_k(s, n_kc)
 inline int tile_cap(const svoo_shape* s, int n_qc, int block_q) {
   return (s->N + block_q - 1) / block_q + groups_q(s, n_qc);
 }
-// cluster count padded for the scoring MMA: a multiple of 32, since scores are
-// read back from TMEM 32 columns at a time
-inline int pad32(int c) { return (c + 31) / 32 * 32; }
+// cluster count padded for the scoring MMA: a multiple of 64, since two
+// threads share a score row and each reads its half from TMEM 32 columns at a time
+inline int pad64(int c) { return (c + 63) / 64 * 64; }
 
 // Bump allocator over a caller-provided workspace (256-byte aligned pieces).
 struct Carver {
