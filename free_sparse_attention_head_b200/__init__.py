@@ -42,7 +42,7 @@ class Shape(ctypes.Structure):
 
 
 _PLAN_FIELDS = ["kmask", "q_label", "q_sizes", "stats", "q_perm", "q_off", "k_perm", "k_off",
-                "tiles", "tile_count"]
+                "tiles", "tile_count", "units", "unit_count"]
 
 
 class _CPlan(ctypes.Structure):
@@ -141,7 +141,7 @@ class Plan:
     """Device buffers of one call's sparse plan (see svoo_plan in include/svoo.h)."""
 
     def __init__(self, shape: Shape, cfg: Config, device):
-        counts = (ctypes.c_int64 * 10)()
+        counts = (ctypes.c_int64 * 12)()
         _check(load().svoo_plan_counts(ctypes.byref(shape), cfg.n_qc, cfg.n_kc, cfg.block_q, counts),
                "svoo_plan_counts")
         self.shape = shape
@@ -177,6 +177,10 @@ class Plan:
     def tile_cap(self) -> int:
         return (self.shape.N + self.cfg.block_q - 1) // self.cfg.block_q + self.Gq
 
+    @property
+    def unit_cap(self) -> int:
+        return (self.shape.N + 255) // 256 + self.Gq
+
     def views(self) -> dict:
         """Per-head views of the plan arrays (still on the device)."""
         BH, N = self.BH, self.shape.N
@@ -191,6 +195,8 @@ class Plan:
             k_off=self.k_off.view(BH, self.Gk + 1),
             tiles=self.tiles.view(BH, self.tile_cap, 4),
             tile_count=self.tile_count.view(BH),
+            units=self.units.view(BH, self.unit_cap, 4),
+            unit_count=self.unit_count.view(BH),
         )
 
 

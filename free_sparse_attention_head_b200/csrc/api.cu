@@ -46,7 +46,7 @@ extern "C" const char* svoo_status_string(svoo_status s) {
 extern "C" int svoo_version(void) { return (0 << 16) | 1; }
 
 extern "C" svoo_status svoo_plan_counts(const svoo_shape* shape, int n_qc, int n_kc, int block_q,
-                                        int64_t counts[10]) {
+                                        int64_t counts[12]) {
   if (!shape_ok(shape) || !counts) return SVOO_ERR_INVALID_ARG;
   if (n_qc < 1 || n_qc > 256 || n_kc < 1 || n_kc > 256) return SVOO_ERR_INVALID_ARG;
   if (block_q != 64 && block_q != 128) return SVOO_ERR_INVALID_ARG;
@@ -62,5 +62,7 @@ extern "C" svoo_status svoo_plan_counts(const svoo_shape* shape, int n_qc, int n
   counts[7] = BH * (Gk + 1);                            // k_off
   counts[8] = BH * tile_cap(shape, n_qc, block_q) * 4;  // tiles
   counts[9] = BH;                                       // tile_count
+  counts[10] = BH * unit_cap(shape, n_qc) * 4;          // units
+  counts[11] = BH;                                      // unit_count
   return SVOO_OK;
 }

@@ -34,6 +34,11 @@ inline int tile_cap(const svoo_shape* s, int n_qc, int block_q) {
 }
 // cluster count padded for the scoring MMA: a multiple of 64, since two
 // threads share a score row and each reads its half from TMEM 32 columns at a time
+// attention work units: up to 256 rows of one query group
+constexpr int kUnitRows = 256;
+inline int unit_cap(const svoo_shape* s, int n_qc) {
+  return (s->N + kUnitRows - 1) / kUnitRows + groups_q(s, n_qc);
+}
 inline int pad64(int c) { return (c + 63) / 64 * 64; }
 
 // Bump allocator over a caller-provided workspace (256-byte aligned pieces).

@@ -8,7 +8,8 @@
 //               with __match_any_sync -- so ties keep token order and the
 //               result is deterministic.
 // tiles_kernel  query tiles of at most block_q rows per group, in (group,
-//               tile) order, with the group's kept key length.
+//               tile) order, with the group's kept key length; and the
+//               attention work units (up to 256 rows of one group).
 // gather_kernel dst[p] = src[perm[p]] row copies (16-byte vectors).
 #include "common.cuh"
 #include "internal.h"
@@ -89,8 +90,9 @@ __global__ void __launch_bounds__(kSortWarps * 32)
 __global__ void tiles_kernel(const int32_t* __restrict__ q_off, const int32_t* __restrict__ k_off,
                              const uint64_t* __restrict__ kmask, int Gq, int Gk, int W, int cap,
                              int block_q, int32_t* __restrict__ tiles,
-                             int32_t* __restrict__ tile_count) {
-  __shared__ int nt[kMaxGroups], base[kMaxGroups], kvl[kMaxGroups];
+                             int32_t* __restrict__ tile_count, int ucap, int32_t* __restrict__ units,
+                             int32_t* __restrict__ unit_count) {
+  __shared__ int nt[kMaxGroups], base[kMaxGroups], kvl[kMaxGroups], nu[kMaxGroups], ubase[kMaxGroups];
   const int h = blockIdx.x, tid = threadIdx.x;
   const int32_t* qo = q_off + static_cast<size_t>(h) * (Gq + 1);
   const int32_t* ko = k_off + static_cast<size_t>(h) * (Gk + 1);
@@ -98,6 +100,7 @@ __global__ void tiles_kernel(const int32_t* __restrict__ q_off, const int32_t* _
   for (int g = tid; g < Gq; g += blockDim.x) {
     int n = qo[g + 1] - qo[g];
     nt[g] = (n + block_q - 1) / block_q;
+    nu[g] = (n + kUnitRows - 1) / kUnitRows;
     int L = 0;
     for (int b = 0; b < Gk; ++b)
       if ((km[g * W + b / 64] >> (b % 64)) & 1ull) L += ko[b + 1] - ko[b];
@@ -105,12 +108,15 @@ __global__ void tiles_kernel(const int32_t* __restrict__ q_off, const int32_t* _
   }
   __syncthreads();
   if (tid == 0) {
-    int run = 0;
+    int run = 0, urun = 0;
     for (int g = 0; g < Gq; ++g) {
       base[g] = run;
       run += nt[g];
+      ubase[g] = urun;
+      urun += nu[g];
     }
     tile_count[h] = min(run, cap);
+    unit_count[h] = min(urun, ucap);
   }
   __syncthreads();
   int32_t* th = tiles + static_cast<size_t>(h) * cap * 4;
@@ -123,6 +129,15 @@ __global__ void tiles_kernel(const int32_t* __restrict__ q_off, const int32_t* _
       th[slot * 4 + 1] = qo[g] + t * block_q;
       th[slot * 4 + 2] = min(block_q, n - t * block_q);
       th[slot * 4 + 3] = kvl[g];
+    }
+    int32_t* uh = units + static_cast<size_t>(h) * ucap * 4;
+    for (int u = 0; u < nu[g]; ++u) {
+      const int slot = ubase[g] + u;
+      if (slot >= ucap) break;
+      uh[slot * 4 + 0] = g;
+      uh[slot * 4 + 1] = qo[g] + u * kUnitRows;
+      uh[slot * 4 + 2] = min(kUnitRows, n - u * kUnitRows);
+      uh[slot * 4 + 3] = kvl[g];
     }
   }
 }
@@ -156,7 +171,7 @@ extern "C" svoo_status svoo_permute(const svoo_shape* shape, const void* q, cons
   if (!shape_ok(shape) || !q || !k || !v || !k_assign || !plan || !qp || !kp || !vp)
     return SVOO_ERR_INVALID_ARG;
   if (!plan->kmask || !plan->q_label || !plan->q_perm || !plan->q_off || !plan->k_perm ||
-      !plan->k_off || !plan->tiles || !plan->tile_count)
+      !plan->k_off || !plan->tiles || !plan->tile_count || !plan->units || !plan->unit_count)
     return SVOO_ERR_INVALID_ARG;
   if (n_qc < 1 || n_qc > 256 || n_kc < 1 || n_kc > 256) return SVOO_ERR_INVALID_ARG;
   if (block_q != 64 && block_q != 128) return SVOO_ERR_INVALID_ARG;
@@ -171,7 +186,8 @@ extern "C" svoo_status svoo_permute(const svoo_shape* shape, const void* q, cons
                                                       plan->k_off, dev_err);
   tiles_kernel<<<BH, 256, 0, st>>>(plan->q_off, plan->k_off, plan->kmask, Gq, Gk, W,
                                    tile_cap(shape, n_qc, block_q), block_q, plan->tiles,
-                                   plan->tile_count);
+                                   plan->tile_count, unit_cap(shape, n_qc), plan->units,
+                                   plan->unit_count);
   const long long rows = static_cast<long long>(BH) * N;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);

@@ -81,7 +81,8 @@ typedef struct {
 /* Device buffers of one call's sparse plan; every array is caller-allocated
  * with the element counts that svoo_plan_counts returns. BH = B*H,
  * Gq = n_qc + (n_text > 0), Gk = n_kc + (n_text > 0), W = ceil(Gk / 64),
- * Tcap = ceil(N / block_q) + Gq. All int32 unless stated. */
+ * Tcap = ceil(N / block_q) + Gq, Ucap = ceil(N / 256) + Gq. All int32 unless
+ * stated. */
 typedef struct {
     uint64_t *kmask;     /* [BH][Gq][W] bit b of row a: query group a attends key group b.
                             Written by svoo_build_mask (after tail merging). */
@@ -96,11 +97,15 @@ typedef struct {
     int32_t *k_off;      /* [BH][Gk+1] */
     int32_t *tiles;      /* [BH][Tcap][4] query tile: group, start position, rows, kv length */
     int32_t *tile_count; /* [BH] tiles in use per head */
+    int32_t *units;      /* [BH][Ucap][4] attention work units: up to 256 consecutive rows of
+                            one query group (two 128-row MMA tiles sharing every key/value
+                            tile): group, start position, rows, kv length (svoo_permute) */
+    int32_t *unit_count; /* [BH] units in use per head */
 } svoo_plan;
 
 /* Element counts of the svoo_plan arrays (in field order) for a shape. */
 svoo_status svoo_plan_counts(const svoo_shape *shape, int n_qc, int n_kc, int block_q,
-                             int64_t counts[10]);
+                             int64_t counts[12]);
 
 /* ------------------------------------------------------------------ clustering
  * Bytes of device workspace svoo_cluster / svoo_cluster_step need. */

@@ -104,6 +104,15 @@ def inject_plan(plan, plans, src_of_head):
         t[:n, 3] = L[p["tiles"][:, 0]]
         V["tiles"][h].copy_(dev(t))
         V["tile_count"][h] = n
+        u = np.zeros((plan.unit_cap, 4), dtype=np.int32)
+        nu = 0
+        for g in range(len(p["q_off"]) - 1):  # attention work units: 256 rows of one group
+            ng = int(p["q_off"][g + 1] - p["q_off"][g])
+            for s0 in range(0, ng, 256):
+                u[nu] = (g, p["q_off"][g] + s0, min(256, ng - s0), L[g])
+                nu += 1
+        V["units"][h].copy_(dev(u))
+        V["unit_count"][h] = nu
 
 
 def gather_by_plan(q, k, v, plans, src_of_head):

@@ -52,13 +52,14 @@ def _shape(B=1, H=2, N=1024, d=64, n_text=0):
 
 def test_plan_counts(lib):
     sh = _shape(N=1000, d=128, n_text=24)
-    counts = (ctypes.c_int64 * 10)()
+    counts = (ctypes.c_int64 * 12)()
     assert lib.svoo_plan_counts(ctypes.byref(sh), 16, 70, 64, counts) == 0
     Gq, Gk = 17, 71
     W = (Gk + 63) // 64
     cap = (1000 + 63) // 64 + Gq
+    ucap = (1000 + 255) // 256 + Gq
     assert list(counts) == [2 * Gq * W, 2000, 2 * Gq, 16, 2000, 2 * (Gq + 1), 2000, 2 * (Gk + 1),
-                            2 * cap * 4, 2]
+                            2 * cap * 4, 2, 2 * ucap * 4, 2]
 
 
 @pytest.mark.parametrize("bad", [
@@ -67,7 +68,7 @@ def test_plan_counts(lib):
 ])
 def test_bad_shapes_rejected(lib, bad):
     sh = _shape(**bad)
-    counts = (ctypes.c_int64 * 10)()
+    counts = (ctypes.c_int64 * 12)()
     assert lib.svoo_plan_counts(ctypes.byref(sh), 16, 16, 64, counts) == 1
     assert lib.svoo_cluster_workspace_size(ctypes.byref(sh), 16, 16) == 0
 
@@ -92,7 +93,7 @@ def test_compute_entry_points_validate_before_launch(lib):
     # workspace too small
     assert lib.svoo_cluster(ctypes.byref(sh), fake, fake, 16, 16, 10, 0, fake, fake, fake, fake, fake,
                             fake, fake, ws - 1024, None, None) == 2
-    plan = svoo._CPlan(*([0x1000] * 10))
+    plan = svoo._CPlan(*([0x1000] * 12))
     mws = lib.svoo_mask_workspace_size(ctypes.byref(sh), 16, 16)
     args = [ctypes.byref(sh), fake, fake, fake, fake, fake, fake, 16, 16]
     assert lib.svoo_build_mask(*args, 2, 64, 2, 0.125, ctypes.byref(plan), fake, mws, None, None) == 1

@@ -252,7 +252,7 @@ def _permute_case(w, q, k, v, plans, src):
     inject_plan(plan, plans, src)
     V = plan.views()
     # clear what permute must produce
-    for f in ("q_perm", "q_off", "k_perm", "k_off", "tiles", "tile_count"):
+    for f in ("q_perm", "q_off", "k_perm", "k_off", "tiles", "tile_count", "units", "unit_count"):
         V[f].fill_(-7)
     k_assign = dev(np.stack([plans[s]["k_label"][:w.n_video] for s in src]))
     qd, kd, vd = qkv_tensors(q, k, v, 1, BH)
@@ -268,11 +268,13 @@ def _permute_case(w, q, k, v, plans, src):
     ref = svoo.Plan(sh, _cfg(w), "cuda")
     inject_plan(ref, plans, src)
     R = ref.views()
-    for f in ("q_perm", "q_off", "k_perm", "k_off", "tile_count"):
+    for f in ("q_perm", "q_off", "k_perm", "k_off", "tile_count", "unit_count"):
         assert torch.equal(V[f], R[f]), (w.name, f)
-    for h in range(BH):  # slots past tile_count are unspecified
+    for h in range(BH):  # slots past the counts are unspecified
         n = int(R["tile_count"][h].item())
         assert torch.equal(V["tiles"][h][:n], R["tiles"][h][:n]), (w.name, "tiles", h)
+        n = int(R["unit_count"][h].item())
+        assert torch.equal(V["units"][h][:n], R["units"][h][:n]), (w.name, "units", h)
     return plan, qp, kp, vp
 
 
