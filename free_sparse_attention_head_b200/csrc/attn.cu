@@ -44,7 +44,7 @@ constexpr float kRescaleLog2 = 8.0f;
 struct AttnSmem {
   uint64_t q_full;
   uint64_t k_full[2], v_full[2], k_empty[2], v_empty[2];
-  uint64_t s_full[2], p_full[2];
+  uint64_t s_full[2], p_half[2], p_full[2];
   uint64_t o_done, mma_final;
   uint32_t tmem_base;
   int abort;
@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(smem_u32(&S->k_empty[s]), 1);
       mbar_init(smem_u32(&S->v_empty[s]), 1);
       mbar_init(smem_u32(&S->s_full[s]), 1);
+      mbar_init(smem_u32(&S->p_half[s]), 128);
       mbar_init(smem_u32(&S->p_full[s]), 128);
     }
     mbar_init(smem_u32(&S->o_done), 1);
@@ -250,17 +251,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int st = j & 1, pst = (j - 1) & 1;
         if (j < nkv) ok = mbar_wait(smem_u32(&S->k_full[st]), (j >> 1) & 1, abort);
         for (int t = 0; t < ntile && ok; ++t) {
-          if (j >= 1) {  // O_t += P_t(j-1) V_{j-1}, P from TMEM
-            ok = mbar_wait(smem_u32(&S->p_full[t]), (j - 1) & 1, abort);
+          if (j >= 1) {  // O_t += P_t(j-1) V_{j-1}, P from TMEM, in two halves of 64 keys
+            ok = mbar_wait(smem_u32(&S->p_half[t]), (j - 1) & 1, abort);
             if (ok && t == 0) ok = mbar_wait(smem_u32(&S->v_full[pst]), ((j - 1) >> 1) & 1, abort);
-            if (!ok) break;
-            tc_fence_after();
+            for (int hf = 0; hf < 2 && ok; ++hf) {
+              if (hf == 1) ok = mbar_wait(smem_u32(&S->p_full[t]), (j - 1) & 1, abort);
+              if (!ok) break;
+              tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < kKvRows / 16; ++kk) {
-              const uint64_t bd = sw128_desc(v_u + pst * kTileBytes + kk * 16 * 128, kKvRows * 128, 1024);
-              umma_f16_ts(tmem + kTmemO0 + t * 128, tmem + kTmemS0 + t * 128 + kPOff + kk * 8, bd, idesc_o,
-                          (j > 1 || kk > 0) ? 1u : 0u);
+              for (int k4 = 0; k4 < kKvRows / 32; ++k4) {
+                const int kk = hf * (kKvRows / 32) + k4;
+                const uint64_t bd = sw128_desc(v_u + pst * kTileBytes + kk * 16 * 128, kKvRows * 128, 1024);
+                umma_f16_ts(tmem + kTmemO0 + t * 128, tmem + kTmemS0 + t * 128 + kPOff + kk * 8, bd, idesc_o,
+                            (j > 1 || kk > 0) ? 1u : 0u);
+              }
             }
+            if (!ok) break;
           }
           if (j < nkv) {  // S_t(j) = Q_t K_j^T
             tc_fence_after();
@@ -293,62 +299,85 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     ChunkCursor cur;
     bool ok = nkv > 0;
     for (int j = 0; j < nkv && ok; ++j) {
+      // validity of tile j's chunks, worked out before waiting for S_t(j); it is
+      // the same for every row, so the masking branch below is warp-uniform
+      int vmask[kChunksPerTile];
+      bool full = true;
+#pragma unroll
+      for (int c8 = 0; c8 < kChunksPerTile; ++c8) {
+        int row_unused;
+        cur.at(S, j * kChunksPerTile + c8, 0, row_unused, vmask[c8]);
+        full = full && vmask[c8] == kChunkRows;
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S->s_full[t]), j & 1, abort));
       if (!ok) break;
       tc_fence_after();
       float s[kKvRows];
+      // all four loads in flight, then one wait that carries the registers
+      tmem_ld32f(lane_base + s_col, s);
+      tmem_ld32f(lane_base + s_col + 32, s + 32);
+      tmem_ld32f(lane_base + s_col + 64, s + 64);
+      tmem_ld32f(lane_base + s_col + 96, s + 96);
+      tmem_wait_ld_f(s);
+      tmem_wait_ld_f(s + 32);
+      tmem_wait_ld_f(s + 64);
+      tmem_wait_ld_f(s + 96);
+      if (!full) {  // a key group's last, partial chunk: invalid keys get -inf (P = 0)
 #pragma unroll
-      for (int q = 0; q < kKvRows / 32; ++q) {
-        uint32_t v[32];
-        tmem_ld32(lane_base + s_col + q * 32, v);
-        tmem_wait_ld();
+        for (int c8 = 0; c8 < kChunksPerTile; ++c8)
 #pragma unroll
-        for (int c = 0; c < 32; ++c) s[q * 32 + c] = __uint_as_float(v[c]);
+          for (int c = 0; c < kChunkRows; ++c)
+            if (c >= vmask[c8]) s[c8 * kChunkRows + c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max (raw scores; scale_log2 > 0 keeps the order), 8 independent chains
+      float m8[8];
 #pragma unroll
-      for (int c8 = 0; c8 < kChunksPerTile; ++c8) {
-        int row_unused, valid;
-        cur.at(S, j * kChunksPerTile + c8, 0, row_unused, valid);
+      for (int e = 0; e < 8; ++e) m8[e] = s[e];
 #pragma unroll
-        for (int c = 0; c < kChunkRows; ++c) {
-          const int col = c8 * kChunkRows + c;
-          s[col] = c < valid ? s[col] * scale_log2 : -INFINITY;
-          mx = fmaxf(mx, s[col]);
-        }
-      }
-      // running max: moved only when it grows by more than 2^8 (P stays <= 2^8)
+      for (int c = 8; c < kKvRows; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale_log2;
+      // running max (log2 units): moved only when it grows by more than 2^8 (P stays <= 2^8)
       const bool grow = mx > m + kRescaleLog2;
       const float alpha = (j > 0 && grow) ? ex2_approx(m - mx) : 1.f;
       if (grow || j == 0) m = fmaxf(m, mx);
-      // P = 2^(s - m), packed bf16 pairs into the upper half of S_t's columns
-      float rs = 0.f;
+      const float neg_m = -m;
+      // P = 2^(s scale_log2 - m), packed bf16 pairs into the upper half of S_t's
+      // columns; the first 64 keys are released to the MMA before the rest
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2_approx(s[q * 32 + 2 * c] - m);
-          const float p1 = ex2_approx(s[q * 32 + 2 * c + 1] - m);
-          rs += p0 + p1;
+          const float p0 = ex2_approx(fmaf(s[q * 32 + 2 * c], scale_log2, neg_m));
+          const float p1 = ex2_approx(fmaf(s[q * 32 + 2 * c + 1], scale_log2, neg_m));
+          rs4[c & 3] += p0 + p1;
           pk[c] = pack_bf16x2(p0, p1);
         }
         tmem_st16(lane_base + s_col + kPOff + q * 16, pk);
-      }
-      l = l * alpha + rs;
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // O_t is stable: S_t(j) completed after PV_t(j-1) in the MMA order, and
-        // PV_t(j) waits for this warpgroup's arrival below
+        if (q == 1) {
+          if (j > 0 && __any_sync(0xffffffffu, grow)) {
+            // rescale this warp's rows of O_t before any of P_t(j) is released (the
+            // first P half is only stored so far): O_t is stable, since S_t(j)
+            // completed after PV_t(j-1) in the MMA order
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + o_col + q * 32, v);
-          tmem_wait_ld();
+            for (int qo = 0; qo < D / 16; ++qo) {
+              uint32_t v[16];
+              tmem_ld16(lane_base + o_col + qo * 16, v);
+              tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * alpha);
-          tmem_st32(lane_base + o_col + q * 32, v);
+              for (int c = 0; c < 16; ++c) v[c] = __float_as_uint(__uint_as_float(v[c]) * alpha);
+              tmem_st16(lane_base + o_col + qo * 16, v);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(smem_u32(&S->p_half[t]));
         }
       }
+      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      l = l * alpha + rs;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&S->p_full[t]));

@@ -310,6 +310,7 @@ def _attn_case(w, q, k, v, plans, src, rows_per_head, heads_checked, seed=0):
         ref, psum, nk = oracle.attn_rows(q[h], k[h], v[h], scale, p["q_label"], p["k_label"], p["kmask"], rows)
         ma, fr = check_attention(o[h][rows], ref, f"{w.name} head {h}")
         worst = (max(worst[0], ma), max(worst[1], fr))
+    print(f"attention {w.name}: worst max-abs {worst[0]:.3e}, worst rel-Frobenius {worst[1]:.3e}")
     return worst
 
 
