@@ -291,20 +291,19 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 //                       last term a 16-wide K chunk of ones against -kappa_j/2
 //                       split into three bf16 parts, so u_j = x.nu_j - kappa_j/2
 //                       and the score is kappa_j - 2 x.nu_j = -2 u_j.
-//   scorers (warps 1-8) thread (row r, column half): |x|^2 over half of the
+//   scorers (warps 8-15) thread (row r, column half): |x|^2 over half of the
 //                       dimensions (then the X buffer goes back), the half's
 //                       maximum of u, and, with the row maximum U and the error
 //                       bound E, its candidates u_j >= U - 2E (they contain the
 //                       exact argmin of the score; then the accumulator goes
 //                       back). A row with one candidate takes it; the others
 //                       are deferred with their candidate list.
-//   summers (warps 9-15) the tile's 8-row blocks, round robin: member sums of
-//                       the labelled rows in fp64 (rows re-read from L2), one
-//                       atomic per run of equal labels in token order, and
-//                       the deferred rows, decided by an fp64 re-score of
-//                       their candidates (ties to the smaller j).
-// Sums of bf16 values with components below 2^-24 dropped are exact in fp64,
-// so the order of the atomic additions does not matter.
+//   summers (warps 1-7) warp w owns rows [128(w-1)/7, 128w/7) of every tile:
+//                       member sums of the labelled rows (re-read from L2), a
+//                       run of equal labels in token order summed in fp32 and
+//                       added with one vector atomic per lane, and the deferred
+//                       rows, decided from the shared-memory nu copies or, inside
+//                       that bound, by an fp64 re-score (ties to the smaller j).
 //
 // Error bound: nu_hi + nu_lo equals nu to 2^-18 relative and the three kappa
 // parts give kappa to 2^-26; the MMA's fp32 accumulation of 2d + 3 exact
@@ -314,6 +313,9 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 
 constexpr int kScorerWarps = 8;
 constexpr int kSummerWarps = 7;
+// warp 0 is the producer; the summers take the next warp ids, the scorers the last
+constexpr int kFirstSummer = 1;
+constexpr int kFirstScorer = kFirstSummer + kSummerWarps;
 constexpr int kAssignWarps = 1 + kScorerWarps + kSummerWarps;
 constexpr int kAssignThreads = kAssignWarps * 32;
 constexpr int kScorers = kScorerWarps * 32;
@@ -337,6 +339,7 @@ struct AssignSmem {
   int16_t cand[2][kTileRows][kHalfCand];
   // published per tile parity for the summers
   int16_t lab[2][kTileRows];               // label; -1 not a video token; -2 deferred
+  uint32_t defmask[2][kTileRows / 32];     // deferred rows of the tile, one bit per row
   int8_t def_n[2][kTileRows];              // deferred row: candidates listed (0 = all)
   int16_t def_cand[2][kTileRows][2 * kHalfCand];
 };
@@ -435,7 +438,7 @@ __device__ __forceinline__ float approx_t(int j, float x0, float x1, float x2, f
 }
 
 template <int D, int CP>
-__device__ int decide_deferred(const AssignSmem* S, int b, int rr, uint32_t xa, uint32_t xb,
+__device__ __noinline__ int decide_deferred(const AssignSmem* S, int b, int rr, uint32_t xa, uint32_t xb,
                                const uint8_t* nuh, const uint8_t* nul, const uint8_t* kparts,
                                float max_nrm, float max_kap, const double* __restrict__ nu_h,
                                const double* __restrict__ kap_h, int C, int lane) {
@@ -666,10 +669,10 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         }
       }
       __syncwarp();
-    } else if (warp <= kScorerWarps) {
+    } else if (warp >= kFirstScorer) {
       // ------------------------------------------------------------ scorers
       const int lq = warp & 3;                   // TMEM lane quarter
-      const int hf = (warp - 1) >> 2;            // column half
+      const int hf = (warp - kFirstScorer) >> 2;  // column half
       const int r = lq * 32 + lane;              // tile row
       const int pair_bar = 1 + lq;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
@@ -740,12 +743,20 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
             tmem_ld32f(ta + 32 * (c + 1), v1);
             tmem_wait_ld_f(v0);
             tmem_wait_ld_f(v1);
-            uint32_t bw[2] = {0u, 0u};
+            // eight independent partial masks per word keep the OR chains short
+            uint32_t p0[8], p1[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              p0[u] = 0u;
+              p1[u] = 0u;
+            }
 #pragma unroll
             for (int q = 0; q < 32; ++q) {
-              bw[0] |= (v0[q] >= thr ? 1u : 0u) << q;
-              bw[1] |= (v1[q] >= thr ? 1u : 0u) << q;
+              p0[q & 7] |= (v0[q] >= thr ? 1u : 0u) << q;
+              p1[q & 7] |= (v1[q] >= thr ? 1u : 0u) << q;
             }
+            uint32_t bw[2] = {((p0[0] | p0[1]) | (p0[2] | p0[3])) | ((p0[4] | p0[5]) | (p0[6] | p0[7])),
+                              ((p1[0] | p1[1]) | (p1[2] | p1[3])) | ((p1[4] | p1[5]) | (p1[6] | p1[7]))};
 #pragma unroll
             for (int w2 = 0; w2 < 2; ++w2) {
               while (bw[w2]) {
@@ -788,6 +799,9 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
             }
           }
           S->lab[b][r] = static_cast<int16_t>(L);
+          // one word per 32 rows: the hf == 0 warps own rows 32 lq .. 32 lq + 31
+          const uint32_t dm = __ballot_sync(0xffffffffu, L == -2);
+          if (lane == 0) S->defmask[b][lq] = dm;
           mbar_arrive(smem_u32(&S->l_full[b]));
         }
       }
@@ -795,7 +809,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       // ------------------------------------------------------------ summers
       // warp sw owns the contiguous rows [r0, r1) of every tile; all of them
       // are fetched with one batch of loads, one tile ahead
-      const int sw = warp - 1 - kScorerWarps;
+      const int sw = warp - kFirstSummer;
       const int r0 = kTileRows * sw / kSummerWarps, r1 = kTileRows * (sw + 1) / kSummerWarps;
       const int nr = r1 - r0;
       const float max_nrm = S->max_nrm, max_kap = S->max_kap;
@@ -850,11 +864,15 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           }
           if (cur >= 0) flush();
         }
-        // deferred rows
+        // deferred rows (usually none: the scorers' bitmask says which)
+        const uint64_t dm64 = (static_cast<uint64_t>(S->defmask[b][(r0 >> 5) + 1 < kTileRows / 32 ? (r0 >> 5) + 1 : (r0 >> 5)]) << 32) |
+                              S->defmask[b][r0 >> 5];
+        uint32_t mine = static_cast<uint32_t>(dm64 >> (r0 & 31)) & ((nr >= 32 ? 0u : (1u << nr)) - 1u);
 #pragma unroll 1
-        for (int k = 0; k < nr; ++k) {
+        while (mine) {
+          const int k = __ffs(mine) - 1;
+          mine &= mine - 1;
           const int rr = r0 + k;
-          if (S->lab[b][rr] != -2) continue;
           uint32_t xa = 0u, xb = 0u;  // this row's words (a dynamic pick from the batch)
 #pragma unroll
           for (int q = 0; q < kSumRows; ++q)

@@ -126,10 +126,14 @@ size_t svoo_cluster_workspace_size(const svoo_shape *shape, int n_qc, int n_kc);
  * Assignment: argmin_j (x - mu_j)^T M (x - mu_j), ties to the smaller j, where
  * M is the normalised second moment of the other side's clusters (identity in
  * the cold first query step); M, nu_j = M mu_j and kappa_j = mu_j . nu_j in
- * fp64. Scores come from tcgen05 bf16 MMAs; when more than one cluster lies
- * within the MMA's error bound of the best, those candidates are re-scored in
- * fp64, so the result is that of an fp64 evaluation. Update: member means from exact fp64
- * sums, rounded once to fp32; an empty cluster keeps its centroid. */
+ * fp64. Scores come from tcgen05 MMAs against nu split into two bf16 rows
+ * (with kappa folded in); when more than one cluster lies within the MMA's
+ * error bound of the best, those candidates are compared again, closer, and
+ * in fp64 when still within bound, so the result is that of an fp64
+ * evaluation. Update: member means from fp32 sums (see the limits above; the
+ * rounding of the sums follows the order of the atomic additions, so two
+ * runs can differ in the last bits of a centroid); an empty cluster keeps its
+ * centroid. */
 svoo_status svoo_cluster(const svoo_shape *shape, const void *q, const void *k, int n_qc,
                          int n_kc, int iters, int warm, int32_t *q_assign, int32_t *k_assign,
                          float *q_cent, float *k_cent, int32_t *q_sizes, int32_t *k_sizes,
