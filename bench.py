@@ -131,6 +131,53 @@ def _rank_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
+def _reduce_max_sum(ms, work, device):
+    """Across the ranks (every rank calls it): the largest time and the summed
+    work, so the whole-job rate is (work of all ranks) / (slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms), float(work)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    f = torch.tensor([float(work)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(f.item())
+
+
+def _rank_seed(seed, rank):
+    """Each rank runs its own batch element: the workload seed shifted by the rank."""
+    return seed + rank
+
+
+TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                            "sparse_attn_wan14b_traffic.json")
+
+
+def _attn_source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    root = os.path.join(os.path.dirname(os.path.abspath(__file__)), "free_sparse_attention_head_b200", "csrc")
+    for name in ("attn.cu", "common.cuh"):
+        with open(os.path.join(root, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _attn_traffic(flops):
+    """DRAM bytes of one attention launch from a committed ncu capture of a
+    smaller case, scaled by the algorithmic FLOPs; None when the capture is
+    absent or the kernel's source changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_sha256") != _attn_source_digest():
+        return None
+    return rec["dram_bytes"] * flops / rec["alg_flops"]
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 
 
@@ -223,7 +270,7 @@ def run_gpu(args):
 
     w = workload.get(WORKLOAD)
     import dataclasses
-    w = dataclasses.replace(w, seed=w.seed + rank)  # this rank's own batch element
+    w = dataclasses.replace(w, seed=_rank_seed(w.seed, rank))  # this rank's own batch element
     if args.heads:
         w = dataclasses.replace(w, H=args.heads)
     q, k, v = workload.make_qkv(w)
@@ -285,18 +332,14 @@ def run_gpu(args):
         dist.barrier()
     clocks = sampler.stop()
     svoo.check_device_errors(err)
-    total_ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms, job_flops = _reduce_max_sum(t_start.elapsed_time(t_end), flops, dev)
     ms_step = total_ms / args.steps
     stage = np.array([[evs[s][i].elapsed_time(evs[s][i + 1]) for i in range(4)] for s in range(args.steps)])
     stage_ms = stage.mean(0)
     attn_ms = float(stage_ms[3])
     burst, sustained, hbm, peak_src = _peaks()
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = job_flops / (ms_step * 1e-3) / 1e12
 
     # dense self-path (keep = 1.0): same library, every cluster pair kept
     dense_plan = svoo.Plan(sh, cfg, dev)
@@ -331,12 +374,8 @@ def run_gpu(args):
         oh.copy_(o_dev, non_blocking=True)
     a1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = a0.elapsed_time(a1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms, _ = _reduce_max_sum(a0.elapsed_time(a1) / e2e_steps, flops, dev)
+    e2e_val = job_flops / (e2e_ms * 1e-3) / 1e12
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -353,7 +392,7 @@ def run_gpu(args):
             "config": _config(w, world),
             "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128>",
                          "achieved": attn_tflops, "peak": sustained, "unit": "TFLOP/s",
-                         "frac": attn_tflops / sustained, "traffic": None,
+                         "frac": attn_tflops / sustained, "traffic": _attn_traffic(flops),
                          "peak_kind": f"bf16 sustained ({peak_src}); kernel timed inside a long step loop",
                          "frac_of_burst_peak": attn_tflops / burst,
                          "alg_flops_per_launch": flops},
