@@ -126,8 +126,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(smem_u32(&S->k_empty[s]), 1);
       mbar_init(smem_u32(&S->v_empty[s]), 1);
       mbar_init(smem_u32(&S->s_full[s]), 1);
-      mbar_init(smem_u32(&S->p_half[s]), 128);
-      mbar_init(smem_u32(&S->p_full[s]), 128);
+      mbar_init(smem_u32(&S->p_half[s]), 4);  // one arrival per softmax warp of the tile
+      mbar_init(smem_u32(&S->p_full[s]), 4);
     }
     mbar_init(smem_u32(&S->o_done), 1);
     mbar_init(smem_u32(&S->mma_final), 1);
@@ -375,14 +375,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(smem_u32(&S->p_half[t]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&S->p_half[t]));
         }
       }
       const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       l = l * alpha + rs;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&S->p_full[t]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S->p_full[t]));
     }
     // ---------------------------------------------------------------- epilogue
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S->o_done), 0, abort));

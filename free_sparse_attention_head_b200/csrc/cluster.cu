@@ -539,11 +539,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     S->abort = 0;
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&S->x_full[b]), 1);
-      mbar_init(smem_u32(&S->x_free[b]), kScorers);
+      // one arrival per warp (after __syncwarp), not per thread
+      mbar_init(smem_u32(&S->x_free[b]), kScorerWarps);
       mbar_init(smem_u32(&S->t_full[b]), 1);
-      mbar_init(smem_u32(&S->t_free[b]), kScorers);
-      mbar_init(smem_u32(&S->l_full[b]), kScorers / 2);
-      mbar_init(smem_u32(&S->l_free[b]), kSummers);
+      mbar_init(smem_u32(&S->t_free[b]), kScorerWarps);
+      mbar_init(smem_u32(&S->l_full[b]), kScorerWarps / 2);
+      mbar_init(smem_u32(&S->l_free[b]), kSummerWarps);
     }
     fence_mbar_init();
     tma_prefetch_desc(&xmap);
@@ -702,7 +703,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           }
           S->xq[hf][r] = (a0 + a1) + (a2 + a3);
         }
-        mbar_arrive(smem_u32(&S->x_free[b]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&S->x_free[b]));
         // pass 1: maximum of this half's u
         const uint32_t ta = lane_base + b * CP + hf * kHalfCols;
         float mx = -INFINITY;
@@ -772,7 +774,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           for (int q = 0; q < kHalfCand; ++q) S->cand[hf][r][q] = cl[q];
         }
         tc_fence_before();
-        mbar_arrive(smem_u32(&S->t_free[b]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&S->t_free[b]));
         named_sync(pair_bar, 64);
         // the row's decision, published for the summers
         if (hf == 0) {
@@ -802,7 +805,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           // one word per 32 rows: the hf == 0 warps own rows 32 lq .. 32 lq + 31
           const uint32_t dm = __ballot_sync(0xffffffffu, L == -2);
           if (lane == 0) S->defmask[b][lq] = dm;
-          mbar_arrive(smem_u32(&S->l_full[b]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&S->l_full[b]));
         }
       }
     } else {
@@ -891,7 +895,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
                        __uint_as_float(xa & 0xffff0000u), __uint_as_float(xb << 16),
                        __uint_as_float(xb & 0xffff0000u), lane);
         }
-        mbar_arrive(smem_u32(&S->l_free[b]));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&S->l_free[b]));
         return true;
       };
       if (t0 < t1) fetch(t0, wa0, wb0);
