@@ -281,7 +281,9 @@ __global__ void __launch_bounds__(1024)
   __shared__ uint64_t msk[256][kMaxW];
   __shared__ int sz[256], nsz[256], rep[256], tl[256], nearv[256];
   __shared__ int mv_donor[128], mv_recv[128], mv_cnt[128];
-  __shared__ int n_moves, st_ident, st_r[2], st_moved, tiles_before;
+  __shared__ int slot_of[256], quota[128];
+  __shared__ int wcnt[32][128];  // per warp of a chunk: tokens of each move's donor
+  __shared__ int n_moves, st_ident, st_r[2], st_moved, tiles_before, left;
   const int h = blockIdx.x, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
   const int rows = Cq + (has_text ? 1 : 0);
@@ -291,6 +293,7 @@ __global__ void __launch_bounds__(1024)
     sz[a] = q_sizes_in[h * Cq + a];
     nsz[a] = 0;
   }
+  for (int a = tid; a < 256; a += blockDim.x) slot_of[a] = -1;
   if (tid == 0) {
     st_ident = 0;
     st_r[0] = st_r[1] = 0;
@@ -372,19 +375,48 @@ __global__ void __launch_bounds__(1024)
       atomicAdd(&st_moved, cnt);
     }
     __syncthreads();
-    // move the donors' highest-index tail tokens; one warp per move
-    for (int m = warp; m < n_moves; m += nwarps) {
-      const int donor = mv_donor[m], recv = mv_recv[m], cnt = mv_cnt[m];
-      int moved = 0;
-      for (int base = nv - 1; base >= 0 && moved < cnt; base -= 32) {
-        int i = base - lane;
-        bool hit = i >= 0 && lab[i] == donor;
-        unsigned bal = __ballot_sync(0xffffffffu, hit);
-        int before = __popc(bal & ((1u << lane) - 1u));
-        if (hit && before < cnt - moved) lab[i] = recv;
-        moved += min(__popc(bal), cnt - moved);
-      }
+    // move the donors' highest-index tail tokens: one backward pass over the
+    // labels in chunks of blockDim.x tokens serves every move of the round;
+    // thread t of a chunk holds the chunk's t-th highest token, so a token's
+    // rank among its donor's tokens is the count in earlier warps plus the
+    // count in earlier lanes of its own warp
+    const int nm = n_moves;
+    for (int m = tid; m < nm; m += blockDim.x) {
+      slot_of[mv_donor[m]] = m;
+      quota[m] = mv_cnt[m];
     }
+    __syncthreads();
+    for (int top = nv - 1; top >= 0; top -= blockDim.x) {
+      if (tid == 0) left = 0;
+      for (int e = tid; e < nwarps * nm; e += blockDim.x) wcnt[e / nm][e % nm] = 0;
+      __syncthreads();
+      const int i = top - tid;
+      int sl = -1;
+      if (i >= 0) {
+        const int l = lab[i];
+        if (l >= 0 && l < Cq) sl = slot_of[l];
+      }
+      if (sl >= 0 && quota[sl] == 0) sl = -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, sl);
+      const int rank_w = __popc(peers & ((1u << lane) - 1u));
+      if (sl >= 0 && rank_w == 0) wcnt[warp][sl] = __popc(peers);
+      __syncthreads();
+      if (sl >= 0) {
+        int before = rank_w;
+        for (int w2 = 0; w2 < warp; ++w2) before += wcnt[w2][sl];
+        if (before < quota[sl]) lab[i] = mv_recv[sl];
+      }
+      __syncthreads();
+      for (int m = tid; m < nm; m += blockDim.x) {
+        int tot = 0;
+        for (int w2 = 0; w2 < nwarps; ++w2) tot += wcnt[w2][m];
+        quota[m] = max(0, quota[m] - tot);
+        if (quota[m] > 0) left = 1;
+      }
+      __syncthreads();
+      if (!left) break;
+    }
+    for (int m = tid; m < nm; m += blockDim.x) slot_of[mv_donor[m]] = -1;
     __syncthreads();
   }
   for (int e = tid; e < Cq * W; e += blockDim.x) km[e] = msk[e / W][e % W];
