@@ -24,7 +24,7 @@ import torch
 __all__ = [
     "Config", "Shape", "Plan", "load", "lib_path", "cluster", "cluster_step", "build_mask",
     "permute", "sparse_attn", "sparse_attention", "check_device_errors", "workspace_sizes",
-    "SvooError",
+    "SvooError", "CLUSTER_WARM", "CLUSTER_IDENTITY",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -128,6 +128,7 @@ class Config:
     select_mode: int = 0          # 0 keep ratio, 1 top-p
     merge_rounds: int = 2
     scale: Optional[float] = None  # default 1/sqrt(d)
+    metric: int = 0               # 0 QK interaction (co-clustering), 1 identity (independent)
 
 
 def make_shape(q: torch.Tensor, n_text: int = 0) -> Shape:
@@ -222,6 +223,16 @@ def check_device_errors(dev_err: torch.Tensor):
         raise SvooError("device error: " + ", ".join(n for b, n in names.items() if v & b))
 
 
+CLUSTER_WARM = 1
+CLUSTER_IDENTITY = 2
+
+
+def _cluster_flags(cfg: Config, warm) -> int:
+    if cfg.metric not in (0, 1):
+        raise SvooError(f"Config.metric must be 0 (QK interaction) or 1 (identity), not {cfg.metric}")
+    return (CLUSTER_WARM if warm is not None else 0) | (CLUSTER_IDENTITY if cfg.metric == 1 else 0)
+
+
 def cluster(q, k, cfg: Config, n_text=0, warm=None, workspace=None, dev_err=None, stream=None):
     """Co-clusters the video tokens of every head; returns a dict of device tensors."""
     _need_cuda(q, k)
@@ -244,7 +255,7 @@ def cluster(q, k, cfg: Config, n_text=0, warm=None, workspace=None, dev_err=None
         out["k_sizes"].copy_(warm[2])
     err = _err_buf(dev_err, dev)
     _check(load().svoo_cluster(ctypes.byref(sh), _ptr(q), _ptr(k), cfg.n_qc, cfg.n_kc, cfg.iters,
-                               int(warm is not None), _ptr(out["q_assign"]), _ptr(out["k_assign"]),
+                               _cluster_flags(cfg, warm), _ptr(out["q_assign"]), _ptr(out["k_assign"]),
                                _ptr(out["q_cent"]), _ptr(out["k_cent"]), _ptr(out["q_sizes"]),
                                _ptr(out["k_sizes"]), _ptr(workspace), workspace.numel(), _ptr(err),
                                _stream(stream)), "svoo_cluster")

@@ -1070,15 +1070,18 @@ extern "C" svoo_status svoo_cluster_step(const svoo_shape* shape, const void* x,
 }
 
 extern "C" svoo_status svoo_cluster(const svoo_shape* shape, const void* q, const void* k, int n_qc,
-                                    int n_kc, int iters, int warm, int32_t* q_assign,
+                                    int n_kc, int iters, int flags, int32_t* q_assign,
                                     int32_t* k_assign, float* q_cent, float* k_cent,
                                     int32_t* q_sizes, int32_t* k_sizes, void* workspace,
                                     size_t workspace_bytes, int32_t* dev_err, void* stream) {
   if (!shape_ok(shape) || !q || !k || !q_assign || !k_assign || !q_cent || !k_cent || !q_sizes ||
       !k_sizes || !workspace)
     return SVOO_ERR_INVALID_ARG;
-  if (!cluster_counts_ok(n_qc) || !cluster_counts_ok(n_kc) || iters < 1 || (warm != 0 && warm != 1))
+  if (!cluster_counts_ok(n_qc) || !cluster_counts_ok(n_kc) || iters < 1 ||
+      (flags & ~(SVOO_CLUSTER_WARM | SVOO_CLUSTER_IDENTITY)) != 0)
     return SVOO_ERR_INVALID_ARG;
+  const bool warm = (flags & SVOO_CLUSTER_WARM) != 0;
+  const bool identity = (flags & SVOO_CLUSTER_IDENTITY) != 0;
   if (!aligned(q, 16) || !aligned(k, 16)) return SVOO_ERR_INVALID_ARG;
   const int BH = bh_of(shape), d = shape->d, N = shape->N, nv = nvideo_of(shape);
   StepWs w;
@@ -1091,11 +1094,12 @@ extern "C" svoo_status svoo_cluster(const svoo_shape* shape, const void* q, cons
   }
   const int Cmax = n_qc > n_kc ? n_qc : n_kc;
   for (int it = 0; it < iters; ++it) {
-    const bool ident = (it == 0 && !warm);
+    const bool ident = identity || (it == 0 && !warm);
     svoo_status s = run_step(shape, q, n_qc, q_cent, q_sizes, q_assign, ident ? nullptr : k_cent,
                              k_sizes, n_kc, w, dev_err, st, it == 0 ? Cmax : 0);
     if (s != SVOO_OK) return s;
-    s = run_step(shape, k, n_kc, k_cent, k_sizes, k_assign, q_cent, q_sizes, n_qc, w, dev_err, st, 0);
+    s = run_step(shape, k, n_kc, k_cent, k_sizes, k_assign, identity ? nullptr : q_cent, q_sizes,
+                 n_qc, w, dev_err, st, 0);
     if (s != SVOO_OK) return s;
   }
   return SVOO_OK;

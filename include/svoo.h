@@ -113,19 +113,29 @@ svoo_status svoo_plan_counts(const svoo_shape *shape, int n_qc, int n_kc, int bl
  * Bytes of device workspace svoo_cluster / svoo_cluster_step need. */
 size_t svoo_cluster_workspace_size(const svoo_shape *shape, int n_qc, int n_kc);
 
+#define SVOO_CLUSTER_WARM 1
+#define SVOO_CLUSTER_IDENTITY 2
+
 /* Co-clusters the video tokens of every head.
  *  q, k      : bf16 [B,H,N,d] (only the first N - n_text tokens are clustered).
  *  iters     : rounds of (query step, key step), each an assignment + update.
- *  warm      : 0 = start from the tokens at floor(j*Nv/C) with a feature-space
- *              first query step; 1 = start from q_cent, k_cent, k_sizes as
- *              given (e.g. the previous timestep's), first query step under
- *              the key-cluster metric.
+ *  flags     : bitwise OR of
+ *              SVOO_CLUSTER_WARM: start from q_cent, k_cent, k_sizes as given
+ *                (e.g. the previous timestep's), first query step under the
+ *                key-cluster metric; without it, start from the tokens at
+ *                floor(j*Nv/C) with a feature-space first query step;
+ *              SVOO_CLUSTER_IDENTITY: every step in feature space (M = I):
+ *                plain k-means of queries and keys separately, the
+ *                independent Euclidean clustering (SVG2's) that iCATS sec. 3.1
+ *                and App. D (Table 3) compare the co-clustering against.
+ *              Any other bit is SVOO_ERR_INVALID_ARG.
  *  q_assign, k_assign : int32 [BH][N - n_text] cluster of every video token.
  *  q_cent, k_cent     : fp32 [BH][n_qc|n_kc][d] centroids (in/out).
  *  q_sizes, k_sizes   : int32 [BH][n_qc|n_kc] members per cluster (k_sizes in/out).
  * Assignment: argmin_j (x - mu_j)^T M (x - mu_j), ties to the smaller j, where
  * M is the normalised second moment of the other side's clusters (identity in
- * the cold first query step); M, nu_j = M mu_j and kappa_j = mu_j . nu_j in
+ * the cold first query step, and in every step under SVOO_CLUSTER_IDENTITY);
+ * M, nu_j = M mu_j and kappa_j = mu_j . nu_j in
  * fp64. Scores come from tcgen05 MMAs against nu split into two bf16 rows
  * (with kappa folded in); when more than one cluster lies within the MMA's
  * error bound of the best, those candidates are compared again, closer, and
@@ -135,7 +145,7 @@ size_t svoo_cluster_workspace_size(const svoo_shape *shape, int n_qc, int n_kc);
  * runs can differ in the last bits of a centroid); an empty cluster keeps its
  * centroid. */
 svoo_status svoo_cluster(const svoo_shape *shape, const void *q, const void *k, int n_qc,
-                         int n_kc, int iters, int warm, int32_t *q_assign, int32_t *k_assign,
+                         int n_kc, int iters, int flags, int32_t *q_assign, int32_t *k_assign,
                          float *q_cent, float *k_cent, int32_t *q_sizes, int32_t *k_sizes,
                          void *workspace, size_t workspace_bytes, int32_t *dev_err,
                          void *stream);

@@ -136,8 +136,10 @@ def update(x, labels, cent_old):
     return cent, sizes
 
 
-def cluster(q, k, n_qc, n_kc, iters, warm=None):
-    """One head. warm = (q_cent, k_cent, k_sizes) start state, or None."""
+def cluster(q, k, n_qc, n_kc, iters, warm=None, identity=False):
+    """One head. warm = (q_cent, k_cent, k_sizes) start state, or None;
+    identity = True clusters queries and keys independently (M = I in every
+    step)."""
     q = _c(q, np.uint16)
     k = _c(k, np.uint16)
     n, d = q.shape
@@ -152,7 +154,8 @@ def cluster(q, k, n_qc, n_kc, iters, warm=None):
         qc = np.array(warm[0], dtype=np.float32, copy=True)
         kc = np.array(warm[1], dtype=np.float32, copy=True)
         ks[:] = warm[2]
-    lib().oracle_cluster(_p(q), _p(k), n, d, n_qc, n_kc, iters, int(warm is not None),
+    flags = int(warm is not None) | (2 if identity else 0)
+    lib().oracle_cluster(_p(q), _p(k), n, d, n_qc, n_kc, iters, flags,
                          _p(qa), _p(ka), _p(qc), _p(kc), _p(qs), _p(ks))
     return dict(q_assign=qa, k_assign=ka, q_cent=qc, k_cent=kc, q_sizes=qs, k_sizes=ks)
 

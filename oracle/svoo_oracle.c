@@ -199,11 +199,15 @@ void oracle_update(const uint16_t *x, int n, int d, const int32_t *assign, int C
 /* step uses the metric of the current key clusters, and each key step uses  */
 /* the metric of the query clusters it has just updated. `iters` rounds of   */
 /* (query step, key step), each step one assignment and one update.          */
-/* warm != 0: q_cent, k_cent and k_sizes hold a start state (e.g. the        */
-/* previous timestep's clusters) and round 0's query step uses M_K too.      */
+/* flags bit 0 (warm): q_cent, k_cent and k_sizes hold a start state (e.g.  */
+/* the previous timestep's clusters) and round 0's query step uses M_K too.  */
+/* flags bit 1 (identity): every step uses M = I, i.e. queries and keys are  */
+/* clustered independently in feature space, the Euclidean clustering that   */
+/* [iCATS] 3.1 and App. D (Table 3) compare against.                         */
 void oracle_cluster(const uint16_t *q, const uint16_t *k, int n, int d, int Cq, int Ck, int iters,
-                    int warm, int32_t *q_assign, int32_t *k_assign, float *q_cent, float *k_cent,
+                    int flags, int32_t *q_assign, int32_t *k_assign, float *q_cent, float *k_cent,
                     int32_t *q_sizes, int32_t *k_sizes) {
+    const int warm = flags & 1, identity = (flags >> 1) & 1;
     double *M = (double *)malloc(sizeof(double) * (size_t)d * d);
     float *tmp = (float *)malloc(sizeof(float) * (size_t)(Cq > Ck ? Cq : Ck) * d);
     if (!warm) {
@@ -211,11 +215,11 @@ void oracle_cluster(const uint16_t *q, const uint16_t *k, int n, int d, int Cq, 
         oracle_init_centroids(k, n, d, Ck, k_cent);
     }
     for (int it = 0; it < iters; ++it) {
-        oracle_metric(k_cent, k_sizes, Ck, d, (it == 0 && !warm), M);
+        oracle_metric(k_cent, k_sizes, Ck, d, identity || (it == 0 && !warm), M);
         oracle_assign(q, n, d, q_cent, Cq, M, q_assign, NULL, NULL);
         oracle_update(q, n, d, q_assign, Cq, q_cent, tmp, q_sizes);
         memcpy(q_cent, tmp, sizeof(float) * (size_t)Cq * d);
-        oracle_metric(q_cent, q_sizes, Cq, d, 0, M);
+        oracle_metric(q_cent, q_sizes, Cq, d, identity, M);
         oracle_assign(k, n, d, k_cent, Ck, M, k_assign, NULL, NULL);
         oracle_update(k, n, d, k_assign, Ck, k_cent, tmp, k_sizes);
         memcpy(k_cent, tmp, sizeof(float) * (size_t)Ck * d);

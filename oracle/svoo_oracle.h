@@ -52,9 +52,10 @@ void oracle_assign(const uint16_t *x, int n, int d, const float *cent, int C, co
 void oracle_update(const uint16_t *x, int n, int d, const int32_t *assign, int C,
                    const float *cent_old, float *cent_new, int32_t *sizes);
 
-/* Full co-clustering of one head: `iters` rounds of (Q step, K step). */
+/* Full co-clustering of one head: `iters` rounds of (Q step, K step).
+ * flags: bit 0 warm start, bit 1 identity metric in every step. */
 void oracle_cluster(const uint16_t *q, const uint16_t *k, int n, int d, int Cq, int Ck, int iters,
-                    int warm, int32_t *q_assign, int32_t *k_assign, float *q_cent, float *k_cent,
+                    int flags, int32_t *q_assign, int32_t *k_assign, float *q_cent, float *k_cent,
                     int32_t *q_sizes, int32_t *k_sizes);
 
 /* Estimated attention mass of every (query cluster, key cluster) pair. fp32. */

@@ -40,6 +40,17 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(svoo.EXPORTS) <= exported
 
 
+def test_cluster_flag_values_match_header():
+    text = open(HEADER).read()
+    macros = dict(re.findall(r"#define (SVOO_CLUSTER_\w+) (\d+)", text))
+    assert int(macros["SVOO_CLUSTER_WARM"]) == svoo.CLUSTER_WARM
+    assert int(macros["SVOO_CLUSTER_IDENTITY"]) == svoo.CLUSTER_IDENTITY
+    assert svoo._cluster_flags(svoo.Config(metric=1), None) == svoo.CLUSTER_IDENTITY
+    assert svoo._cluster_flags(svoo.Config(), (0, 0, 0)) == svoo.CLUSTER_WARM
+    with pytest.raises(svoo.SvooError):
+        svoo._cluster_flags(svoo.Config(metric=2), None)
+
+
 def test_status_strings_and_version(lib):
     assert lib.svoo_status_string(0) == b"ok"
     assert lib.svoo_status_string(2) == b"workspace too small"
@@ -83,9 +94,10 @@ def test_compute_entry_points_validate_before_launch(lib):
     # null inputs
     assert lib.svoo_cluster(ctypes.byref(sh), None, fake, 16, 16, 10, 0, fake, fake, fake, fake, fake,
                             fake, fake, ws, None, None) == 1
-    # cluster counts out of range, iters < 1, bad warm flag
-    for nq, nk, it, warm in [(0, 16, 10, 0), (16, 300, 10, 0), (16, 16, 0, 0), (16, 16, 1, 2)]:
-        assert lib.svoo_cluster(ctypes.byref(sh), fake, fake, nq, nk, it, warm, fake, fake, fake, fake,
+    # cluster counts out of range, iters < 1, unknown flag bits
+    for nq, nk, it, flags in [(0, 16, 10, 0), (16, 300, 10, 0), (16, 16, 0, 0), (16, 16, 1, 4),
+                              (16, 16, 1, -1), (16, 16, 1, 3 | 8)]:
+        assert lib.svoo_cluster(ctypes.byref(sh), fake, fake, nq, nk, it, flags, fake, fake, fake, fake,
                                 fake, fake, fake, ws, None, None) == 1
     # misaligned q
     assert lib.svoo_cluster(ctypes.byref(sh), odd, fake, 16, 16, 10, 0, fake, fake, fake, fake, fake,

@@ -171,24 +171,29 @@ def test_cluster_trajectory(name):
                 kc, ks = new_c, new_s
 
 
+@pytest.mark.parametrize("metric", [0, 1], ids=["interaction", "identity"])
 @pytest.mark.parametrize("name", ["tiny", "ragged"])
-def test_cluster_whole(name):
-    """The whole GPU clustering run against the oracle's run (drift report: the
-    two trajectories may part at an fp32-vs-fp64 near-tie and then drift, so
-    the bound here is loose; the lockstep test above is the hard gate)."""
+def test_cluster_whole(name, metric):
+    """The whole GPU clustering run against the oracle's run, under the QK
+    interaction metric and under the identity flag (independent k-means of
+    each side). Drift report: the two trajectories may part at a near-tie
+    decided by centroids that differ in their last bits and then drift, so the
+    bound here is loose; the lockstep test above is the hard gate."""
     w = SMALL[name]
     q, k, _ = workload.make_qkv(w)
     qd, kd, _ = qkv_tensors(q, k, k, w.B, w.H)
-    cl = svoo.cluster(qd, kd, _cfg(w), n_text=w.n_text)
+    cfg = _cfg(w)
+    cfg.metric = metric
+    cl = svoo.cluster(qd, kd, cfg, n_text=w.n_text)
     torch.cuda.synchronize()
     _err_ok(cl["dev_err"])
     nv = w.n_video
     for h in range(w.B * w.H):
-        o = oracle.cluster(q[h][:nv], k[h][:nv], w.n_qc, w.n_kc, w.iters)
+        o = oracle.cluster(q[h][:nv], k[h][:nv], w.n_qc, w.n_kc, w.iters, identity=metric == 1)
         for side in ("q", "k"):
             g = cl[f"{side}_assign"][h].cpu().numpy()
             agree = (g == o[f"{side}_assign"]).mean()
-            print(f"whole-run drift {name} head {h} {side}: agreement {agree:.5f}")
+            print(f"whole-run drift {name} metric {metric} head {h} {side}: agreement {agree:.5f}")
             assert agree >= 0.98, (name, h, side, agree)
             if agree == 1.0:
                 # same final labels: same sizes; centroids within the drift of

@@ -201,6 +201,68 @@ def test_warm_start_equals_continuation():
         assert np.array_equal(two[key], cont[key]), key
 
 
+def _lloyd(x, init, iters):
+    """Textbook Lloyd iterations in fp64 from `init` (fp32 centroids after each
+    update, an empty cluster keeping its centroid)."""
+    cent = init.astype(np.float32)
+    for _ in range(iters):
+        d2 = ((x[:, None, :] - cent.astype(np.float64)[None]) ** 2).sum(-1)
+        lab = np.argmin(d2, axis=1)
+        cent = np.stack([x[lab == j].mean(0).astype(np.float32) if (lab == j).any() else cent[j]
+                         for j in range(cent.shape[0])])
+    return lab, cent
+
+
+def test_identity_mode_is_independent_lloyd():
+    """Under the identity flag both sides run plain k-means of their own tokens
+    (the independent Euclidean clustering of iCATS sec. 3.1 / App. D): several
+    rounds equal separate textbook Lloyd runs of Q and of K."""
+    rng = np.random.default_rng(11)
+    n, d, Cq, Ck, iters = 160, 8, 6, 5, 3
+    q = _rand_bf16(rng, (n, d), 2.0)
+    k = _rand_bf16(rng, (n, d), 2.0)
+    res = oracle.cluster(q, k, Cq, Ck, iters=iters, identity=True)
+    for side, x_bits, C in (("q", q, Cq), ("k", k, Ck)):
+        x = bf16_bits_to_f32(x_bits).astype(np.float64)
+        assert (np.abs(x)[x != 0] >= 2.0 ** -24).all()   # no component the update drops
+        lab, cent = _lloyd(x, x[[j * n // C for j in range(C)]], iters)
+        assert np.array_equal(res[f"{side}_assign"], lab), side
+        assert np.array_equal(res[f"{side}_cent"], cent), side
+        assert np.array_equal(res[f"{side}_sizes"], np.bincount(lab, minlength=C)), side
+
+
+def test_identity_mode_sides_do_not_interact():
+    """Independent clustering: the key clusters do not depend on the queries
+    (and vice versa), while under the interaction metric they do."""
+    rng = np.random.default_rng(12)
+    n, d, C = 140, 8, 5
+    q = _rand_bf16(rng, (n, d), 2.0)
+    k = _rand_bf16(rng, (n, d), 2.0)
+    q2 = _rand_bf16(rng, (n, d), 2.0)
+    a = oracle.cluster(q, k, C, C, iters=3, identity=True)
+    b = oracle.cluster(q2, k, C, C, iters=3, identity=True)
+    for key in ("k_assign", "k_cent", "k_sizes"):
+        assert np.array_equal(a[key], b[key]), key
+    ca = oracle.cluster(q, k, C, C, iters=3)
+    cb = oracle.cluster(q2, k, C, C, iters=3)
+    assert not np.array_equal(ca["k_assign"], cb["k_assign"])
+
+
+def test_identity_warm_start_is_lloyd_from_given_centroids():
+    rng = np.random.default_rng(13)
+    n, d, C = 120, 6, 4
+    q = _rand_bf16(rng, (n, d), 2.0)
+    k = _rand_bf16(rng, (n, d), 2.0)
+    qc0 = rng.standard_normal((C, d)).astype(np.float32)
+    kc0 = rng.standard_normal((C, d)).astype(np.float32)
+    res = oracle.cluster(q, k, C, C, iters=2, warm=(qc0, kc0, np.zeros(C, np.int32)), identity=True)
+    for side, x_bits, c0 in (("q", q, qc0), ("k", k, kc0)):
+        x = bf16_bits_to_f32(x_bits).astype(np.float64)
+        lab, cent = _lloyd(x, c0, 2)
+        assert np.array_equal(res[f"{side}_assign"], lab), side
+        assert np.array_equal(res[f"{side}_cent"], cent), side
+
+
 # --------------------------------------------------------------------- pair mass / selection
 
 
