@@ -60,6 +60,8 @@ _SIGS = {
     "oracle_tiles": (_I, [_P, _I, _I, _P]),
     "oracle_attn_rows": (None, [_P, _P, _P, _I, _I, _F, _P, _P, _P, _I, _P, _I, _P, _P, _P]),
     "oracle_dense_attn_rows": (None, [_P, _P, _P, _I, _I, _F, _P, _I, _P]),
+    "oracle_psa_attends": (_I, [ctypes.c_longlong, ctypes.c_longlong, ctypes.c_longlong, _P]),
+    "oracle_psa_plan": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
 }
 
 
@@ -273,3 +275,48 @@ def plan_head(q, k, n_qc, n_kc, iters, keep, block_q, n_text=0, mode=0, top_p=0.
                 q_label=q_label, k_label=k_label, nonempty=ne, merge_stats=st,
                 q_perm=q_perm, q_off=q_off, k_perm=k_perm, k_off=k_off,
                 tiles=tiles(q_off, block_q), scale=float(np.float32(scale)))
+
+
+# --------------------------------------------------------------------------- PSA stripe mask
+
+PSA_INF = 2 ** 31 - 1   # stride "infinity": one diagonal band, no wrap-around
+
+
+def psa_params(prm):
+    """(Tw, To, Ts, Sw, So, Ss) with None or math.inf for an infinite stride -> int32[6]."""
+    out = []
+    for i, v in enumerate(prm):
+        if i in (2, 5) and (v is None or v == math.inf):
+            v = PSA_INF
+        out.append(int(v))
+    return np.array(out, dtype=np.int32)
+
+
+def psa_attends(i, j, HW, prm):
+    return bool(lib().oracle_psa_attends(int(i), int(j), int(HW), _p(psa_params(prm))))
+
+
+def psa_plan(T, H, W, block, n_text, prm):
+    """Labels [N], block mask [G, Wd] and block sizes [G] of one head."""
+    bt, bh, bw = block
+    nb = -(-T // bt) * -(-H // bh) * -(-W // bw)
+    G = nb + (1 if n_text > 0 else 0)
+    Wd = (G + 63) // 64
+    N = T * H * W + n_text
+    label = np.empty(N, dtype=np.int32)
+    kmask = np.empty((G, Wd), dtype=np.uint64)
+    sizes = np.empty(G, dtype=np.int32)
+    r = lib().oracle_psa_plan(T, H, W, bt, bh, bw, n_text, _p(psa_params(prm)), _p(label),
+                              _p(kmask), _p(sizes))
+    assert r == nb
+    return dict(label=label, kmask=kmask, sizes=sizes, nb=nb, G=G)
+
+
+def psa_plan_head(T, H, W, block, n_text, prm, block_q):
+    """Oracle of the static stripe-mask path for one head: the PSA plan, then
+    the same permutation and query tiles as the clustered path."""
+    p = psa_plan(T, H, W, block, n_text, prm)
+    q_perm, q_off = permute(p["label"], p["G"])
+    return dict(kmask=p["kmask"], q_label=p["label"], k_label=p["label"], q_sizes=p["sizes"],
+                nb=p["nb"], q_perm=q_perm, q_off=q_off, k_perm=q_perm, k_off=q_off,
+                tiles=tiles(q_off, block_q))

@@ -576,3 +576,60 @@ void oracle_dense_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t
     }
     free(s);
 }
+
+/* [PSA] sec. 3.2, Alg. 1 (mask definition): 1 if position i attends position */
+/* j under M(Tw, To, Ts, Sw, So, Ss) = prm[0..5], the sequence being frames   */
+/* of HW positions. Frame and in-frame index of both, then the inter-frame    */
+/* band test on the frame distance and the intra-frame band test on the       */
+/* in-frame distance. A stride of INT32_MAX stands for infinity: the distance */
+/* never wraps, leaving one diagonal band on that axis.                       */
+int oracle_psa_attends(long long i, long long j, long long HW, const int32_t *prm) {
+    const long long tq = i / HW, sq = i % HW;
+    const long long tk = j / HW, sk = j % HW;
+    const long long dt = tk - tq;
+    if (llabs(dt - prm[1]) % prm[2] > (long long)prm[0] - 1) return 0;
+    const long long ds = sk - sq;
+    return llabs(ds - prm[4]) % prm[5] <= (long long)prm[3] - 1;
+}
+
+/* [PSA] sec. 3.2 (PSABlock; block-centric layout) and Alg. 1: the sparse    */
+/* plan of one head for a static stripe mask. Video tokens lie in (T, H, W)   */
+/* raster order, n_text text tokens follow them. A token's label is its       */
+/* PSABlock (t / bt, y / bh, x / bw), numbered in raster order over the grid  */
+/* (T', H', W') = (ceil(T / bt), ceil(H / bh), ceil(W / bw)); blocks on the   */
+/* far edges are smaller (no padding tokens are made). Text tokens take label */
+/* nb = T'H'W'. Masking is at PSABlock granularity: bit b of row a is Alg. 1  */
+/* with i = a, j = b and HW = H'W' (block distances). The text row attends    */
+/* every group and every row attends the text group. Writes label[N],         */
+/* kmask[G][Wd] (G = nb + (n_text > 0), Wd = ceil(G / 64)) and sizes[G];      */
+/* returns nb.                                                                */
+int oracle_psa_plan(int T, int H, int W, int bt, int bh, int bw, int n_text, const int32_t *prm,
+                    int32_t *label, uint64_t *kmask, int32_t *sizes) {
+    const int Tb = (T + bt - 1) / bt, Hb = (H + bh - 1) / bh, Wb = (W + bw - 1) / bw;
+    const int nb = Tb * Hb * Wb;
+    const int G = nb + (n_text > 0), Wd = (G + 63) / 64;
+    const long long nv = (long long)T * H * W;
+    for (int g = 0; g < G; ++g) sizes[g] = 0;
+    for (long long i = 0; i < nv; ++i) {
+        const int t = (int)(i / ((long long)H * W));
+        const int y = (int)((i / W) % H);
+        const int x = (int)(i % W);
+        const int a = ((t / bt) * Hb + y / bh) * Wb + x / bw;
+        label[i] = a;
+        sizes[a] += 1;
+    }
+    for (int e = 0; e < n_text; ++e) {
+        label[nv + e] = nb;
+        sizes[nb] += 1;
+    }
+    memset(kmask, 0, sizeof(uint64_t) * (size_t)G * Wd);
+    for (int a = 0; a < G; ++a) {
+        for (int b = 0; b < G; ++b) {
+            int keep;
+            if (a == nb || b == nb) keep = 1; /* text row / text column */
+            else keep = oracle_psa_attends(a, b, (long long)Hb * Wb, prm);
+            if (keep) kmask[(size_t)a * Wd + b / 64] |= 1ull << (b % 64);
+        }
+    }
+    return nb;
+}

@@ -16,8 +16,9 @@
  *           and Timestep-Adaptive Sparsity" (paperlayer.ai summary), sections
  *           3.1, 3.3, 4.1, 4.3, appendix E.1 / E.2.
  *   [PSA]   "PSA: Parameterized Stripe Attention" full text, section 2 (SVG2's
- *           k-means clustering, permutation and top-k cluster selection) and
- *           Table 2 (FLOP accounting).
+ *           k-means clustering, permutation and top-k cluster selection),
+ *           section 3.2 with Algorithm 1 (the stripe mask M(Tw,To,Ts,Sw,So,Ss)
+ *           at PSABlock granularity) and Table 2 (FLOP accounting).
  *
  * Readings of points the pages leave open are stated beside each function.
  * Arrays are row-major; bf16 values are passed as their uint16 bit patterns.
@@ -88,6 +89,15 @@ void oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, i
 /* Textbook dense softmax attention for selected query rows (fp64). */
 void oracle_dense_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int n, int d,
                             float scale, const int32_t *rows, int nrows, double *out);
+
+/* [PSA] Alg. 1: does position i attend position j (frames of HW positions)
+ * under M(Tw, To, Ts, Sw, So, Ss) = prm[0..5]; a stride INT32_MAX is infinity. */
+int oracle_psa_attends(long long i, long long j, long long HW, const int32_t *prm);
+
+/* Static stripe-mask plan of one head at PSABlock granularity: labels (the
+ * token's block), block mask and block sizes; returns the block count. */
+int oracle_psa_plan(int T, int H, int W, int bt, int bh, int bw, int n_text, const int32_t *prm,
+                    int32_t *label, uint64_t *kmask, int32_t *sizes);
 
 #ifdef __cplusplus
 }
