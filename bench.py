@@ -14,6 +14,10 @@ Multi-GPU (torchrun): every rank runs its own call (its own batch element,
 weak scaling, no data-path collective); time = max over ranks.
 --impl reference times the CPU oracle (the only reference this path has) on a
 bounded sample of the same workload and extrapolates by algorithmic work.
+
+--mask psa measures the second plan source instead: PSA's static stripe mask
+(svoo_psa_mask -> svoo_permute -> svoo_sparse_attn) on the same call, PSABlock
+3 x 8 x 16, per-head parameters drawn from PSA's Table 7 mix.
 """
 from __future__ import annotations
 
@@ -35,6 +39,7 @@ if ROOT not in sys.path:
 import workload  # noqa: E402
 
 METRIC = "sparse-attn ms/call & effective TFLOPS (% bf16 TC peak) at Wan-14B shape"
+METRIC_PSA = "PSA stripe-mask sparse-attn effective TFLOPS (% bf16 TC peak) at Wan-14B shape"
 WORKLOAD = "wan2.1-14b"
 
 
@@ -46,6 +51,21 @@ def _peaks():
         return float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), float(p["hbm_gbs"]), "measured"
     except Exception:
         return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _config_psa(w, n_gpus, block, params):
+    from collections import Counter
+    fmt = lambda p: "(" + ",".join("inf" if v == math.inf else str(v) for v in p) + ")"
+    top = ", ".join(f"{c} x {n}" for c, n in Counter(fmt(p) for p in params).most_common(3))
+    return {
+        "workload": f"{w.name}: B=1 per GPU, H={w.H}, N={w.N} ({'x'.join(map(str, w.grid))}), d={w.d}, "
+                    f"PSA stripe mask, PSABlock {'x'.join(map(str, block))}, per-head (Tw,To,Ts,Sw,So,Ss) "
+                    f"seeded from PSA Table 7's head-count mix (most frequent here: {top})",
+        "global_batch": n_gpus,
+        "seq_len": w.N,
+        "parallelism": f"independent calls per GPU x{n_gpus}",
+        "l2": "inputs 2.3 GB per GPU > 126 MB L2; no flush between steps",
+    }
 
 
 def _config(w, n_gpus):
@@ -60,9 +80,12 @@ def _config(w, n_gpus):
     }
 
 
-def _launch_count(iters):
+def _launch_count(iters, psa=False):
+    # psa: labels + mask 2; permute 5 (sort, tiles, 3 gathers); attention 1
+    if psa:
+        return 2 + 5 + 1
     # init x2; round 0: q (nu, assign, finalize) + k (m, nu, assign, finalize);
-    # later rounds 4 + 4; mask 3; permute 5 (sort, tiles, 3 gathers); attention 1
+    # later rounds 4 + 4; mask 3; permute 5; attention 1
     return 2 + 7 + 8 * (iters - 1) + 3 + 5 + 1
 
 
@@ -152,6 +175,8 @@ def _rank_seed(seed, rank):
 
 TRAFFIC_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
                             "sparse_attn_wan14b_traffic.json")
+TRAFFIC_FILE_PSA = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                                "sparse_attn_wan14b_psa_traffic.json")
 
 
 def _attn_source_digest():
@@ -164,12 +189,12 @@ def _attn_source_digest():
     return h.hexdigest()
 
 
-def _attn_traffic(flops):
+def _attn_traffic(flops, psa=False):
     """DRAM bytes of one attention launch from a committed ncu capture of a
-    smaller case, scaled by the algorithmic FLOPs; None when the capture is
-    absent or the kernel's source changed since it was taken."""
+    smaller case (of the same plan source), scaled by the algorithmic FLOPs;
+    None when the capture is absent or the kernel's source changed since."""
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(TRAFFIC_FILE_PSA if psa else TRAFFIC_FILE) as f:
             rec = json.load(f)
     except (OSError, ValueError):
         return None
@@ -218,26 +243,66 @@ def cpu_oracle_sample(w, head=0, iters=1, attn_rows=64, seed=0):
                 sample_seconds=t3 - t0)
 
 
+def cpu_oracle_sample_psa(w, block, params, head=0, attn_rows=64, seed=0):
+    """Times the oracle's stripe-mask plan and `attn_rows` attention rows of one
+    head; returns the extrapolated seconds of one full call."""
+    import oracle
+    q, k, v = workload.make_qkv(w, heads=[head])
+    q, k, v = q[0], k[0], v[0]
+    BH = w.B * w.H
+    t0 = time.perf_counter()
+    p = oracle.psa_plan_head(*w.grid, block, w.n_text, params[head], w.block_q)
+    t1 = time.perf_counter()
+    rows = np.sort(np.random.default_rng(seed).choice(w.N, attn_rows, replace=False)).astype(np.int32)
+    _, _, nk = oracle.attn_rows(q, k, v, float(np.float32(1.0 / math.sqrt(w.d))), p["q_label"],
+                                p["k_label"], p["kmask"], rows)
+    t2 = time.perf_counter()
+    full_flops = 0.0
+    for h in range(BH):
+        o = oracle.psa_plan(*w.grid, block, w.n_text, params[h])
+        G = o["G"]
+        bits = (o["kmask"][:, np.arange(G) // 64] >> (np.arange(G) % 64).astype(np.uint64)) & np.uint64(1)
+        L = (bits.astype(np.int64) * o["sizes"][None, :]).sum(1)
+        full_flops += 4.0 * w.d * float((o["sizes"].astype(np.int64) * L).sum())
+    sample_flops = 4.0 * w.d * float(nk.sum())
+    est = (t1 - t0) * BH + (t2 - t1) * (full_flops / max(sample_flops, 1.0))
+    return dict(est_seconds=est, full_flops=full_flops, sample_seconds=t2 - t0,
+                sample=f"1 head of {w.name} (head {head}, {params[head]}): stripe-mask plan + permutation, "
+                       f"{attn_rows} of {w.N} attention rows; extrapolated x{BH} heads, attention by "
+                       f"algorithmic FLOPs")
+
+
 def run_reference(args):
     rank, world, _ = _rank_env()
     if rank != 0:
         return 0
     w = workload.get(WORKLOAD)
+    psa = args.mask == "psa"
+    if psa:
+        block = workload.PSA_BLOCKS[w.name]
+        prm = workload.psa_strategies(w, block)
+
+        def sample(head, rows, seed=0):
+            return cpu_oracle_sample_psa(w, block, prm, head=head, attn_rows=rows, seed=seed)
+    else:
+        def sample(head, rows, seed=0):
+            return cpu_oracle_sample(w, head=head, iters=1, attn_rows=rows, seed=seed)
     for _ in range(args.warmup):
-        cpu_oracle_sample(w, head=0, iters=1, attn_rows=8)
+        sample(0, 8)
     vals, secs = [], []
     cores = 1
     info = None
     for s in range(args.steps):
-        info = cpu_oracle_sample(w, head=s % (w.B * w.H), iters=1, attn_rows=32, seed=s)
+        info = sample(s % (w.B * w.H), 32, seed=s)
         vals.append(info["full_flops"] / info["est_seconds"] / 1e12)
         secs.append(info["est_seconds"])
     value = statistics.median(vals)
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "impl": "reference", "metric": METRIC_PSA if psa else METRIC, "value": value, "unit": "TFLOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": statistics.median(secs) * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(w, world),
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config_psa(w, world, block, prm) if psa else _config(w, world),
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
                          "sample": info["sample"] + " (one step = one such sample)"},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -281,11 +346,19 @@ def run_gpu(args):
 
     qd, kd, vd = as_dev(q), as_dev(k), as_dev(v)
     keep = torch.from_numpy(w.keep_ratios()).to(dev)
-    cfg = svoo.Config(n_qc=w.n_qc, n_kc=w.n_kc, iters=w.iters, block_q=w.block_q)
+    psa = args.mask == "psa"
     sh = svoo.make_shape(qd)
-    cws, mws = svoo.workspace_sizes(sh, cfg)
-    ws_c = torch.empty(cws, dtype=torch.uint8, device=dev)
-    ws_m = torch.empty(mws, dtype=torch.uint8, device=dev)
+    if psa:
+        block = workload.PSA_BLOCKS[w.name]
+        psa_prm = workload.psa_strategies(w, block)
+        params = svoo.psa_params(psa_prm, dev)
+        cfg = svoo.psa_config(w.grid, block, w.block_q)
+        k_assign = torch.empty(BH, w.n_video, dtype=torch.int32, device=dev)
+    else:
+        cfg = svoo.Config(n_qc=w.n_qc, n_kc=w.n_kc, iters=w.iters, block_q=w.block_q)
+        cws, mws = svoo.workspace_sizes(sh, cfg)
+        ws_c = torch.empty(cws, dtype=torch.uint8, device=dev)
+        ws_m = torch.empty(mws, dtype=torch.uint8, device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     plan = svoo.Plan(sh, cfg, dev)
     qp, kp, vp, out = (torch.empty_like(qd) for _ in range(4))
@@ -294,13 +367,20 @@ def run_gpu(args):
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        cl = svoo.cluster(qd, kd, cfg, workspace=ws_c, dev_err=err)
-        if evs:
-            evs[1].record(stream)
-        svoo.build_mask(sh, cl, keep, cfg, plan=plan, workspace=ws_m, dev_err=err)
+        if psa:
+            if evs:
+                evs[1].record(stream)
+            svoo.psa_mask(sh, w.grid, block, params, cfg, plan=plan, k_assign=k_assign, dev_err=err)
+            ka = k_assign
+        else:
+            cl = svoo.cluster(qd, kd, cfg, workspace=ws_c, dev_err=err)
+            if evs:
+                evs[1].record(stream)
+            svoo.build_mask(sh, cl, keep, cfg, plan=plan, workspace=ws_m, dev_err=err)
+            ka = cl["k_assign"]
         if evs:
             evs[2].record(stream)
-        svoo.permute(qd, kd, vd, cl["k_assign"], plan, qp=qp, kp=kp, vp=vp, dev_err=err)
+        svoo.permute(qd, kd, vd, ka, plan, qp=qp, kp=kp, vp=vp, dev_err=err)
         if evs:
             evs[3].record(stream)
         svoo.sparse_attn(qp, kp, vp, plan, out=out, dev_err=err)
@@ -341,11 +421,17 @@ def run_gpu(args):
     attn_tflops = flops / (attn_ms * 1e-3) / 1e12
     value = job_flops / (ms_step * 1e-3) / 1e12
 
-    # dense self-path (keep = 1.0): same library, every cluster pair kept
+    # dense self-path (keep = 1.0, or PSA's full window): same library, every pair kept
     dense_plan = svoo.Plan(sh, cfg, dev)
-    cl = svoo.cluster(qd, kd, cfg, workspace=ws_c, dev_err=err)
-    svoo.build_mask(sh, cl, torch.ones_like(keep), cfg, plan=dense_plan, workspace=ws_m, dev_err=err)
-    svoo.permute(qd, kd, vd, cl["k_assign"], dense_plan, qp=qp, kp=kp, vp=vp, dev_err=err)
+    if psa:
+        Tb, Hb, Wb = (-(-a // b) for a, b in zip(w.grid, block))
+        full = svoo.psa_params([(Tb, 0, math.inf, Hb * Wb, 0, math.inf)] * BH, dev)
+        svoo.psa_mask(sh, w.grid, block, full, cfg, plan=dense_plan, k_assign=k_assign, dev_err=err)
+        svoo.permute(qd, kd, vd, k_assign, dense_plan, qp=qp, kp=kp, vp=vp, dev_err=err)
+    else:
+        cl = svoo.cluster(qd, kd, cfg, workspace=ws_c, dev_err=err)
+        svoo.build_mask(sh, cl, torch.ones_like(keep), cfg, plan=dense_plan, workspace=ws_m, dev_err=err)
+        svoo.permute(qd, kd, vd, cl["k_assign"], dense_plan, qp=qp, kp=kp, vp=vp, dev_err=err)
     svoo.sparse_attn(qp, kp, vp, dense_plan, out=out, dev_err=err)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -370,7 +456,10 @@ def run_gpu(args):
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
-        o_dev, _ = svoo.sparse_attention(qd, kd, vd, keep, cfg, dev_err=err)
+        if psa:
+            o_dev, _ = svoo.psa_attention(qd, kd, vd, w.grid, block, params, block_q=w.block_q, dev_err=err)
+        else:
+            o_dev, _ = svoo.sparse_attention(qd, kd, vd, keep, cfg, dev_err=err)
         oh.copy_(o_dev, non_blocking=True)
     a1.record(stream)
     torch.cuda.synchronize()
@@ -379,25 +468,31 @@ def run_gpu(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        info = cpu_oracle_sample(workload.get(WORKLOAD), head=0, iters=2, attn_rows=256)
+        if psa:
+            info = cpu_oracle_sample_psa(w, block, psa_prm, head=0, attn_rows=256)
+        else:
+            info = cpu_oracle_sample(workload.get(WORKLOAD), head=0, iters=2, attn_rows=256)
         cpu = {"value": info["full_flops"] / info["est_seconds"] / 1e12, "unit": "TFLOPS", "cores": 1,
                "kind": "oracle", "sample": info["sample"],
                "est_ms_per_call": info["est_seconds"] * 1e3, "sample_seconds": info["sample_seconds"]}
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "metric": METRIC_PSA if psa else METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded center-mixture Q/K, Gaussian V)",
-            "config": _config(w, world),
+            "config": _config_psa(w, world, block, psa_prm) if psa else _config(w, world),
             "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel<128>",
                          "achieved": attn_tflops, "peak": sustained, "unit": "TFLOP/s",
-                         "frac": attn_tflops / sustained, "traffic": _attn_traffic(flops),
+                         "frac": attn_tflops / sustained, "traffic": _attn_traffic(flops, psa),
                          "peak_kind": f"bf16 sustained ({peak_src}); kernel timed inside a long step loop",
                          "frac_of_burst_peak": attn_tflops / burst,
                          "alg_flops_per_launch": flops},
-            "stages_ms": {"cluster": float(stage_ms[0]), "mask_merge": float(stage_ms[1]),
-                          "permute": float(stage_ms[2]), "attention": attn_ms},
+            "stages_ms": ({"psa_mask": float(stage_ms[1]), "permute": float(stage_ms[2]),
+                           "attention": attn_ms} if psa else
+                          {"cluster": float(stage_ms[0]), "mask_merge": float(stage_ms[1]),
+                           "permute": float(stage_ms[2]), "attention": attn_ms}),
             "overhead_ratio": float((stage_ms[0] + stage_ms[1]) / attn_ms),
             "dense_self": {"ms": dense_ms, "tflops": dense_flops / (dense_ms * 1e-3) / 1e12,
                            "alg_tflop": dense_flops / 1e12},
@@ -405,7 +500,7 @@ def run_gpu(args):
             "query_tiles_before_after_merge": [int(stats[:, 5].sum()), int(stats[:, 6].sum())],
             "e2e": {"value": e2e_val, "unit": "TFLOPS", "ms_per_call": e2e_ms,
                     "h2d_bytes_per_step": 3 * qd.numel() * 2, "d2h_bytes_per_step": qd.numel() * 2},
-            "gpu_launches": _launch_count(w.iters) * args.steps,
+            "gpu_launches": _launch_count(w.iters, psa) * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
@@ -423,6 +518,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="svoo", choices=["svoo", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mask", default="cluster", choices=["cluster", "psa"],
+                    help="plan source: online co-clustering (default) or PSA's static stripe mask")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the first H heads only (smaller profiling captures; not a bench line)")
     args = ap.parse_args()

@@ -24,7 +24,8 @@ import torch
 __all__ = [
     "Config", "Shape", "Plan", "load", "lib_path", "cluster", "cluster_step", "build_mask",
     "permute", "sparse_attn", "sparse_attention", "check_device_errors", "workspace_sizes",
-    "SvooError", "CLUSTER_WARM", "CLUSTER_IDENTITY",
+    "SvooError", "CLUSTER_WARM", "CLUSTER_IDENTITY", "PSA_INF", "psa_config", "psa_params",
+    "psa_mask", "psa_attention",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -69,6 +70,8 @@ _SIGS = {
                              _P, _P]),
     "svoo_permute": (_I, [_SP, _P, _P, _P, _P, _I, _I, _I, _PP, _P, _P, _P, _P, _P]),
     "svoo_sparse_attn": (_I, [_SP, _P, _P, _P, _PP, _I, _I, _I, _F, _P, _P, _P]),
+    "svoo_psa_block_count": (_I, [_I, _I, _I, _I, _I, _I]),
+    "svoo_psa_mask": (_I, [_SP, _I, _I, _I, _I, _I, _I, _P, _I, _PP, _P, _P, _P]),
 }
 
 EXPORTS = tuple(_SIGS)
@@ -352,3 +355,59 @@ def sparse_attention(q, k, v, keep, cfg: Config, n_text=0, dev_err=None, stream=
     qp, kp, vp = permute(q, k, v, cl["k_assign"], plan, dev_err=err, stream=stream)
     out = sparse_attn(qp, kp, vp, plan, dev_err=err, stream=stream)
     return out, dict(cl=cl, plan=plan, dev_err=err)
+
+
+# --------------------------------------------------------------------------- static stripe mask
+
+PSA_INF = 2 ** 31 - 1   # SVOO_PSA_INF: infinite stride, one diagonal band on that axis
+
+
+def psa_params(per_head, device) -> torch.Tensor:
+    """int32 [B*H, 6] device tensor from per-head (Tw, To, Ts, Sw, So, Ss) tuples;
+    None or math.inf for an infinite stride."""
+    rows = []
+    for prm in per_head:
+        if len(prm) != 6:
+            raise SvooError("a PSA mask has six parameters (Tw, To, Ts, Sw, So, Ss)")
+        rows.append([PSA_INF if (i in (2, 5) and (v is None or v == math.inf)) else int(v)
+                     for i, v in enumerate(prm)])
+    return torch.tensor(rows, dtype=torch.int32).to(device)
+
+
+def psa_config(grid, block, block_q: int = 128, scale: Optional[float] = None) -> Config:
+    """The Config of a stripe-mask plan: one group per PSABlock on each side."""
+    nb = load().svoo_psa_block_count(*grid, *block)
+    if nb < 1 or nb > 256:
+        raise SvooError(f"PSABlock grid of {grid} by {block} has {nb} blocks (1..256 supported)")
+    return Config(n_qc=nb, n_kc=nb, iters=1, block_q=block_q, scale=scale)
+
+
+def psa_mask(shape: Shape, grid, block, params: torch.Tensor, cfg: Config,
+             plan: Optional[Plan] = None, k_assign: Optional[torch.Tensor] = None, dev_err=None,
+             stream=None):
+    """Plan of the PSA stripe mask (svoo_psa_mask): returns (plan, k_assign)."""
+    _need_cuda(params)
+    dev = params.device
+    BH, nv = shape.B * shape.H, shape.N - shape.n_text
+    if tuple(params.shape) != (BH, 6) or params.dtype != torch.int32 or not params.is_contiguous():
+        raise SvooError("params must be a contiguous int32 [B*H, 6] tensor")
+    if plan is None:
+        plan = Plan(shape, cfg, dev)
+    if k_assign is None:
+        k_assign = torch.empty(BH, nv, dtype=torch.int32, device=dev)
+    err = _err_buf(dev_err, dev)
+    _check(load().svoo_psa_mask(ctypes.byref(shape), *grid, *block, _ptr(params), cfg.block_q, plan.c,
+                                _ptr(k_assign), _ptr(err), _stream(stream)), "svoo_psa_mask")
+    return plan, k_assign
+
+
+def psa_attention(q, k, v, grid, block, params: torch.Tensor, n_text=0, block_q: int = 128,
+                  scale: Optional[float] = None, dev_err=None, stream=None):
+    """The stripe-mask path: PSA plan -> permute -> sparse attention."""
+    sh = make_shape(q, n_text)
+    cfg = psa_config(grid, block, block_q, scale)
+    err = _err_buf(dev_err, q.device)
+    plan, k_assign = psa_mask(sh, grid, block, params, cfg, dev_err=err, stream=stream)
+    qp, kp, vp = permute(q, k, v, k_assign, plan, dev_err=err, stream=stream)
+    out = sparse_attn(qp, kp, vp, plan, dev_err=err, stream=stream)
+    return out, dict(plan=plan, k_assign=k_assign, dev_err=err, cfg=cfg)

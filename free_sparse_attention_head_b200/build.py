@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsvoo.so")
-SOURCES = ["api.cu", "cluster.cu", "mask.cu", "permute.cu", "attn.cu"]
+SOURCES = ["api.cu", "cluster.cu", "mask.cu", "permute.cu", "attn.cu", "psa.cu"]
 HEADERS = ["common.cuh", "internal.h"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 

@@ -27,6 +27,11 @@
  *                        kept cluster pairs, online softmax over the kept key
  *                        tiles only, O written back in token order.
  *
+ * A second source of the plan replaces steps 1-2 for heads with a static
+ * pattern: svoo_psa_mask writes the stripe mask of "PSA: Parameterized Stripe
+ * Attention" (section 3.2, Algorithm 1) with every PSABlock as one group;
+ * steps 3-4 then run unchanged.
+ *
  * Conventions shared by every entry point:
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library
  *    never allocates, frees or synchronises. Work is enqueued on `stream` (a
@@ -204,6 +209,45 @@ svoo_status svoo_build_mask(const svoo_shape *shape, const float *q_cent, const 
                             int select_mode, int block_q, int merge_rounds, float scale,
                             const svoo_plan *plan, void *workspace, size_t workspace_bytes,
                             int32_t *dev_err, void *stream);
+
+/* ------------------------------------------------------------------ static stripe mask
+ * Number of PSABlocks, ceil(T/bt) ceil(H/bh) ceil(W/bw), of a token grid; 0
+ * for a non-positive argument. */
+int svoo_psa_block_count(int grid_t, int grid_h, int grid_w, int block_t, int block_h,
+                         int block_w);
+
+#define SVOO_PSA_INF 2147483647 /* stride "infinity": one diagonal band on that axis */
+
+/* The plan of the stripe mask M(Tw, To, Ts, Sw, So, Ss) of PSA ("PSA:
+ * Parameterized Stripe Attention", section 3.2 and Algorithm 1), in place of
+ * svoo_cluster + svoo_build_mask.
+ *  grid_t, grid_h, grid_w : the video tokens form a (T, H, W) grid in raster
+ *        order (T*H*W must equal N - n_text).
+ *  block_t, block_h, block_w : the PSABlock. The block grid is (T', H', W') =
+ *        (ceil(T/bt), ceil(H/bh), ceil(W/bw)), nb = T'H'W' <= 256 blocks,
+ *        numbered in raster order; blocks on the far edges hold only the
+ *        tokens that exist (no padding).
+ *  params : int32 [B*H][6], DEVICE: (Tw, To, Ts, Sw, So, Ss) of each head.
+ *        Tw, Sw >= 0; Ts, Ss >= 1, SVOO_PSA_INF for infinity. A head with a
+ *        parameter out of range gets no video block pair (its text group, if
+ *        any, is still kept) and sets bit 4 in dev_err.
+ *  Masking is at PSABlock granularity: query block a keeps key block b when
+ *  Algorithm 1 holds for the block indices (frame = index / (H'W'), in-frame
+ *  position = index % (H'W')), i.e. the frame distance D satisfies
+ *  (|D - To| mod Ts) <= Tw - 1 and the in-frame distance E satisfies
+ *  (|E - So| mod Ss) <= Sw - 1. Text tokens form group nb, which attends
+ *  every group and which every group attends.
+ *  Writes plan->kmask, q_label (a token's block), q_sizes and stats (kept
+ *  video block pairs, nb, 0, 0, 0, query tiles, query tiles, 0), sized by
+ *  svoo_plan_counts(shape, nb, nb, block_q), and k_assign (int32
+ *  [B*H][N - n_text], the key block of every video token) for svoo_permute.
+ *  Then call svoo_permute and svoo_sparse_attn with n_qc = n_kc = nb: the
+ *  stable sort lays every block's tokens out contiguously in raster order,
+ *  which is PSA's block-centric (T', H', W', bt, bh, bw) layout. */
+svoo_status svoo_psa_mask(const svoo_shape *shape, int grid_t, int grid_h, int grid_w,
+                          int block_t, int block_h, int block_w, const int32_t *params,
+                          int block_q, svoo_plan *plan, int32_t *k_assign, int32_t *dev_err,
+                          void *stream);
 
 /* ------------------------------------------------------------------ permutation
  * Stable counting sorts of the merged query labels (plan->q_label) and of the

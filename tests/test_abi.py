@@ -118,3 +118,26 @@ def test_compute_entry_points_validate_before_launch(lib):
                                 float("nan"), fake, None, None) == 1
     assert lib.svoo_sparse_attn(ctypes.byref(sh), fake, fake, fake, None, 16, 16, 64, 0.125, fake,
                                 None, None) == 1
+
+
+def test_psa_block_count_and_mask_validation(lib):
+    assert lib.svoo_psa_block_count(21, 45, 80, 3, 8, 16) == 7 * 6 * 5
+    assert lib.svoo_psa_block_count(6, 10, 12, 2, 4, 5) == 27
+    assert lib.svoo_psa_block_count(0, 10, 12, 2, 4, 5) == 0
+    assert lib.svoo_psa_block_count(6, 10, 12, 2, 0, 5) == 0
+    sh = _shape(B=1, H=2, N=6 * 10 * 12 + 4, d=128, n_text=4)
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    plan = svoo._CPlan(*([0x1000] * 12))
+    ok = (6, 10, 12, 2, 4, 5)
+    args = lambda grid_block, params=fake, bq=128, pl=ctypes.byref(plan), ka=fake: (
+        ctypes.byref(sh), *grid_block, params, bq, pl, ka, None, None)
+    # grid does not cover the video tokens, too many blocks, bad block, block_q, nulls
+    for gb in [(6, 10, 11, 2, 4, 5), (6, 10, 12, 1, 1, 1), (6, 10, 12, 0, 4, 5)]:
+        assert lib.svoo_psa_mask(*args(gb)) == 1, gb
+    assert lib.svoo_psa_mask(*args(ok, bq=96)) == 1
+    assert lib.svoo_psa_mask(*args(ok, params=None)) == 1
+    assert lib.svoo_psa_mask(*args(ok, ka=None)) == 1
+    assert lib.svoo_psa_mask(*args(ok, pl=None)) == 1
+    empty = svoo._CPlan(*([0] * 12))
+    assert lib.svoo_psa_mask(*args(ok, pl=ctypes.byref(empty))) == 1

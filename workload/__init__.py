@@ -34,7 +34,8 @@ import numpy as np
 
 __all__ = [
     "Workload", "WORKLOADS", "get", "splitmix64", "f32_to_bf16_bits",
-    "bf16_bits_to_f32", "make_qkv", "cell_centers", "sweep_workload",
+    "bf16_bits_to_f32", "make_qkv", "cell_centers", "sweep_workload", "psa_strategies",
+    "PSA_BLOCKS",
 ]
 
 _MASK64 = np.uint64(0xFFFFFFFFFFFFFFFF)
@@ -199,3 +200,49 @@ def sweep_workload(n_tokens: int, keep: float) -> Workload:
 
 def get(name: str) -> Workload:
     return WORKLOADS[name]
+
+
+# --------------------------------------------------------------------------- stripe-mask strategies
+
+# PSABlock per workload for the static stripe mask: 3 x 8 x 16 as the PSA pages
+# use for Wan 2.1 (appendix C.2); the HunyuanVideo grid takes 3 x 16 x 16, since
+# 3 x 8 x 16 would give 330 blocks and the plan holds at most 256 groups.
+PSA_BLOCKS = {"tiny": (2, 4, 4), "wan2.1-1.3b": (3, 8, 16), "wan2.1-14b": (3, 8, 16),
+              "hunyuanvideo-13b": (3, 16, 16)}
+
+# The ten most frequent (Tw, To, Ts), (Sw, So, Ss) of PSA-Search on Wan 2.1 14B
+# (PSA appendix C.3, Table 7) with their head counts; None = the full window,
+# math.inf = an infinite stride. The remaining 27.02% of heads ("all other
+# configurations") are drawn from the candidate ranges of appendix C.2.
+PSA_TABLE7 = (
+    (None, 32000), (((7, 0, math.inf), (3, 0, 3)), 25257), (((1, 0, math.inf), (5, 0, 6)), 11778),
+    (((7, 0, math.inf), (1, 0, 3)), 11069), (((7, 0, math.inf), (3, 0, 1)), 9014),
+    (((7, 0, math.inf), (3, 0, 5)), 6810), (((7, 0, math.inf), (1, 0, 5)), 5655),
+    (((7, 0, math.inf), (5, 0, 3)), 5470), (((1, 0, 3), (5, 0, 6)), 5088),
+    (((3, 0, math.inf), (5, 0, 6)), 4622),
+)
+PSA_OTHER = 43237
+
+
+def psa_strategies(w: Workload, block: Optional[tuple] = None) -> list:
+    """Per-(batch, head) stripe-mask parameters (Tw, To, Ts, Sw, So, Ss) for a
+    workload, drawn (seeded) from the Table 7 head-count distribution, the rest
+    uniformly from the appendix C.2 candidate ranges (Tw in [1, T'), To in
+    {0, +-1, +-2}, Ts in {1, 2, 3, inf}, Sw in [1, W'), So in {0, +-1}, Ss in
+    {1, 3, 5, 6, inf}); the full window is (T', 0, inf, H'W', 0, inf)."""
+    block = block or PSA_BLOCKS[w.name]
+    T, Y, X = w.grid
+    Tb, Yb, Xb = -(-T // block[0]), -(-Y // block[1]), -(-X // block[2])
+    rng = np.random.Generator(np.random.PCG64(w.seed * 1000 + 999_971))
+    counts = np.array([c for _, c in PSA_TABLE7] + [PSA_OTHER], dtype=np.float64)
+    pick = rng.choice(len(counts), size=w.B * w.H, p=counts / counts.sum())
+    out = []
+    for k in pick:
+        if k < len(PSA_TABLE7):
+            cfg = PSA_TABLE7[k][0]
+            out.append((Tb, 0, math.inf, Yb * Xb, 0, math.inf) if cfg is None else cfg[0] + cfg[1])
+        else:
+            out.append((int(rng.integers(1, max(Tb, 2))), int(rng.choice([0, 1, -1, 2, -2])),
+                        [1, 2, 3, math.inf][rng.integers(4)], int(rng.integers(1, max(Xb, 2))),
+                        int(rng.choice([0, 1, -1])), [1, 3, 5, 6, math.inf][rng.integers(5)]))
+    return out
