@@ -251,7 +251,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       bool ok = mbar_wait(smem_u32(&S->q_full), 0, abort);
       for (int j = 0; j <= nkv && ok; ++j) {
         const int st = j & 1, pst = (j - 1) & 1;
-        if (j < nkv) ok = mbar_wait(smem_u32(&S->k_full[st]), (j >> 1) & 1, abort);
         for (int t = 0; t < ntile && ok; ++t) {
           if (j >= 1) {  // O_t += P_t(j-1) V_{j-1}, P from TMEM, in two halves of 64 keys
             ok = mbar_wait(smem_u32(&S->p_half[t]), (j - 1) & 1, abort);
@@ -270,7 +269,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             if (!ok) break;
           }
-          if (j < nkv) {  // S_t(j) = Q_t K_j^T
+          if (j < nkv) {  // S_t(j) = Q_t K_j^T; K_j is waited for after PV_A(j-1) is issued,
+                          // so a late K tile does not hold back the product that is ready
+            if (t == 0) ok = mbar_wait(smem_u32(&S->k_full[st]), (j >> 1) & 1, abort);
+            if (!ok) break;
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
