@@ -13,7 +13,8 @@
 //
 // psa_label_kernel  the block of every token (q_label, and k_assign for the
 //                   video tokens); text tokens take group nb.
-// psa_mask_kernel   one CTA per head: the block mask, block sizes and stats.
+// psa_mask_kernel   one CTA per block-mask row: the row's bits, the block's size,
+//                   and its share of the head's stats.
 #include "common.cuh"
 #include "internal.h"
 
@@ -60,44 +61,42 @@ __device__ __forceinline__ bool psa_attends(long long a, long long b, long long 
 
 __device__ __forceinline__ int edge_extent(int n, int blk, int idx) { return min(blk, n - idx * blk); }
 
-// grid BH, block 256
-__global__ void __launch_bounds__(256)
+// grid (G, BH), block kPsaRowThreads: one CTA per block-mask row a, one thread
+// per key group b (bit b of the row); the warps' ballots are the row's 32-bit
+// halves. Row a also writes its block size and adds its kept video pairs and
+// query tiles to the head's stats (zeroed by the host before the launch).
+constexpr int kPsaRowThreads = 320;  // >= 257 groups, whole 64-bit words
+
+__global__ void __launch_bounds__(kPsaRowThreads)
     psa_mask_kernel(PsaGrid g, const int32_t* __restrict__ params, int n_text, int G, int Wd,
                     int block_q, uint64_t* __restrict__ kmask, int32_t* __restrict__ q_sizes,
                     int32_t* __restrict__ stats, int* __restrict__ err) {
-  __shared__ long long prm[6];
-  __shared__ int kept, tiles;
-  const int h = blockIdx.x, tid = threadIdx.x;
-  if (tid < 6) prm[tid] = params[h * 6 + tid];
-  if (tid == 0) {
-    kept = 0;
-    tiles = 0;
-  }
-  __syncthreads();
+  const int a = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
+  long long prm[6];
+#pragma unroll
+  for (int i = 0; i < 6; ++i) prm[i] = params[h * 6 + i];
   const bool ok = prm[0] >= 0 && prm[3] >= 0 && prm[2] >= 1 && prm[5] >= 1;
-  if (!ok && tid == 0) report_error(err, kErrBadPlan);
+  if (!ok && a == 0 && tid == 0) report_error(err, kErrBadPlan);
   const long long hw = static_cast<long long>(g.Hb) * g.Wb;
-  int my_kept = 0;
-  for (int e = tid; e < G * Wd; e += blockDim.x) {
-    const int a = e / Wd, wd = e - a * Wd;
-    uint64_t bits = 0, video = 0;
-    for (int bb = 0; bb < 64; ++bb) {
-      const int b = wd * 64 + bb;
-      if (b >= G) break;
-      bool keep;
-      if (a == g.nb || b == g.nb) {
-        keep = true;
-      } else {
-        keep = ok && psa_attends(a, b, hw, prm);
-        if (keep) video |= 1ull << bb;
-      }
-      if (keep) bits |= 1ull << bb;
+  const int b = tid;
+  bool keep = false, video = false;
+  if (b < G) {
+    if (a == g.nb || b == g.nb) {
+      keep = true;
+    } else {
+      keep = ok && psa_attends(a, b, hw, prm);
+      video = keep;
     }
-    my_kept += __popcll(video);
-    kmask[(static_cast<size_t>(h) * G + a) * Wd + wd] = bits;
   }
-  int my_tiles = 0;
-  for (int a = tid; a < G; a += blockDim.x) {
+  const unsigned bits = __ballot_sync(0xffffffffu, keep);
+  const unsigned vbits = __ballot_sync(0xffffffffu, video);
+  int32_t* st = stats + static_cast<size_t>(h) * 8;
+  if (lane == 0) {
+    if (warp < 2 * Wd) reinterpret_cast<uint32_t*>(kmask + (static_cast<size_t>(h) * G + a) * Wd)[warp] = bits;
+    if (vbits) atomicAdd(&st[0], __popc(vbits));
+  }
+  if (tid == 0) {
     int n;
     if (a < g.nb) {
       const int x = a % g.Wb, y = (a / g.Wb) % g.Hb, t = a / (g.Wb * g.Hb);
@@ -106,21 +105,12 @@ __global__ void __launch_bounds__(256)
       n = n_text;
     }
     q_sizes[static_cast<size_t>(h) * G + a] = n;
-    my_tiles += (n + block_q - 1) / block_q;
-  }
-  if (my_kept) atomicAdd(&kept, my_kept);
-  if (my_tiles) atomicAdd(&tiles, my_tiles);
-  __syncthreads();
-  if (tid == 0) {
-    int32_t* st = stats + static_cast<size_t>(h) * 8;
-    st[0] = kept;
-    st[1] = g.nb;
-    st[2] = 0;
-    st[3] = 0;
-    st[4] = 0;
-    st[5] = tiles;
-    st[6] = tiles;
-    st[7] = 0;
+    const int tiles = (n + block_q - 1) / block_q;
+    if (tiles) {
+      atomicAdd(&st[5], tiles);
+      atomicAdd(&st[6], tiles);
+    }
+    if (a == 0) st[1] = g.nb;
   }
 }
 
@@ -164,7 +154,11 @@ extern "C" svoo_status svoo_psa_mask(const svoo_shape* shape, int grid_t, int gr
   const int G = groups_q(shape, nb), Wd = mask_words(shape, nb);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   psa_label_kernel<<<dim3((N + 255) / 256, BH), 256, 0, st>>>(g, N, nv, plan->q_label, k_assign);
-  psa_mask_kernel<<<BH, 256, 0, st>>>(g, params, shape->n_text, G, Wd, block_q, plan->kmask,
-                                      plan->q_sizes, plan->stats, dev_err);
+  static_assert(kPsaRowThreads >= kPsaMaxBlocks + 1 && kPsaRowThreads % 64 == 0, "one thread per group");
+  if (cudaMemsetAsync(plan->stats, 0, sizeof(int32_t) * 8 * static_cast<size_t>(BH), st) != cudaSuccess)
+    return SVOO_ERR_CUDA;
+  psa_mask_kernel<<<dim3(G, BH), kPsaRowThreads, 0, st>>>(g, params, shape->n_text, G, Wd, block_q,
+                                                          plan->kmask, plan->q_sizes, plan->stats,
+                                                          dev_err);
   return launch_status();
 }
