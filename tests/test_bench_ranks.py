@@ -10,6 +10,8 @@ import socket
 import subprocess
 import sys
 
+import pytest
+
 import bench
 from _ranks import reduction_rank
 
@@ -53,13 +55,14 @@ def test_reference_arm_is_silent_off_rank_zero():
     assert r.stdout.strip() == ""
 
 
-def test_reference_line_shape():
+@pytest.mark.parametrize("mask", ["cluster", "psa"])
+def test_reference_line_shape(mask):
     """Rank 0 of the reference arm prints one JSON line with the contract's keys
-    (one bounded oracle sample, a few seconds of CPU)."""
+    (one bounded oracle sample, a few seconds of CPU), for either plan source."""
     env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
-                       timeout=600)
+                        "--mask", mask, "--steps", "1", "--warmup", "0"], env=env,
+                       capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
     assert len(lines) == 1
@@ -70,3 +73,4 @@ def test_reference_line_shape():
         assert key in line, key
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert ("PSA" in line["metric"]) == (mask == "psa")

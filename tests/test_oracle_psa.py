@@ -146,3 +146,20 @@ def test_table7_configurations_on_the_wan_grid():
     p = oracle.psa_plan(*grid, block, 0, (1, 0, INF, 5, 0, 6))
     want = (t[None] == t[:, None]) & (np.abs(s[None] - s[:, None]) % 6 < 5)
     assert np.array_equal(_bits(p["kmask"], p["G"]), want)
+
+
+def test_seeded_strategies_are_deterministic_and_in_range():
+    """The workload's per-head stripe parameters: the same draw every time,
+    widths and strides in the appendix C.2 ranges, Table 7 rows or the full
+    window on the Wan 2.1 14B block grid."""
+    import workload
+    w = workload.get("wan2.1-14b")
+    a = workload.psa_strategies(w)
+    assert a == workload.psa_strategies(w) and len(a) == w.B * w.H
+    table7 = {c[0] + c[1] for c, _ in workload.PSA_TABLE7 if c is not None}
+    full = (7, 0, INF, 30, 0, INF)
+    for prm in a:
+        Tw, To, Ts, Sw, So, Ss = prm
+        assert 1 <= Tw <= 7 and To in (0, 1, -1, 2, -2) and Ts in (1, 2, 3, INF)
+        assert 1 <= Sw <= 30 and So in (0, 1, -1) and Ss in (1, 3, 5, 6, INF)
+        assert prm in table7 or prm == full or (Tw < 7 and Sw < 5)
