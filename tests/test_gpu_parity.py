@@ -7,7 +7,8 @@ another GPU stage) and its outputs are compared with the oracle's:
   trajectory (the GPU step started from the oracle's exact state): labels
   agree on >= 99.9% of tokens and every disagreement sits where the oracle's
   own fp64 distances are within 1e-4 (relative); with full agreement the
-  centroids and sizes are bit-exact;
+  sizes are exact and every centroid lies within the bound of its fp32 member
+  sums, (n + 18) 2^-24 mean|x| + 2^-24 + 1 ulp of the oracle's;
 * whole clustering run on the GPU alone: a drift report against the oracle's
   run (>= 98%; the trajectories may part at a near-tie);
 * mask + tail merge, permutation, query tiles, gathered copies: bit-exact;
@@ -17,7 +18,8 @@ another GPU stage) and its outputs are compared with the oracle's:
 
 The Wan2.1-14B case runs all 40 heads in one call, as the benchmark does, and
 checks sampled heads / rows; other heads receive copies of the sampled heads'
-oracle inputs.
+oracle inputs. The sweep points cover the shortest sequence at the sparsest
+keep ratio and the longest (131,072 tokens) at the dense one, Zipf-skewed.
 """
 import math
 
@@ -438,3 +440,19 @@ def test_hunyuan_text_tokens():
     _mask_case(w, plans, heads, 0, keeps)
     _permute_case(w, q, k, v, plans, heads)
     _attn_case(w, q, k, v, plans, heads, 512, heads)
+
+
+@pytest.mark.parametrize("n_tokens,keep", [(8192, 0.05), (131072, 1.0)])
+def test_sweep_points(n_tokens, keep):
+    """Sweep/stress shape (H = 24 in the sweep; the first 2 heads here), Zipf-skewed
+    cluster sizes, at the shortest sequence with the sparsest keep ratio and at
+    the longest sequence with the dense keep ratio: mask, permutation and
+    attention on sampled rows against the oracle's plans."""
+    w = _sub(workload.sweep_workload(n_tokens, keep), 2)
+    q, k, v = workload.make_qkv(w)
+    heads = [0, 1]
+    keeps = w.keep_ratios()
+    plans = oracle_plan_heads(w, q, k, heads, keeps, iters=2)
+    _mask_case(w, plans, heads, 0, keeps)
+    _permute_case(w, q, k, v, plans, heads)
+    _attn_case(w, q, k, v, plans, heads, 128, heads)
