@@ -72,7 +72,7 @@ float oracle_exp(float x) {
 /* quadratic form in the original feature space. Replacing a query q by its   */
 /* centroid mu changes q.k by (q - mu).k for every key k; the mean squared    */
 /* change over the keys is (q - mu)^T M (q - mu) with M = E_k[k k^T]. With    */
-/* keys summarised by their clusters ("the previous key-cluster metric"):     */
+/* keys summarised by their clusters (the key clusters of the step before):   */
 /*     M = sum_b n_b c_b c_b^T / sum_b n_b.                                   */
 /* The key step uses the same form with the query clusters. identity != 0     */
 /* gives M = I (plain feature-space k-means, [iCATS] 4.1's first step).       */

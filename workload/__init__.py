@@ -212,8 +212,8 @@ PSA_BLOCKS = {"tiny": (2, 4, 4), "wan2.1-1.3b": (3, 8, 16), "wan2.1-14b": (3, 8,
 
 # The ten most frequent (Tw, To, Ts), (Sw, So, Ss) of PSA-Search on Wan 2.1 14B
 # (PSA appendix C.3, Table 7) with their head counts; None = the full window,
-# math.inf = an infinite stride. The remaining 27.02% of heads ("all other
-# configurations") are drawn from the candidate ranges of appendix C.2.
+# math.inf = an infinite stride. The remaining 27.02% of heads (the table's
+# remainder row) are drawn from the candidate ranges of appendix C.2.
 PSA_TABLE7 = (
     (None, 32000), (((7, 0, math.inf), (3, 0, 3)), 25257), (((1, 0, math.inf), (5, 0, 6)), 11778),
     (((7, 0, math.inf), (1, 0, 3)), 11069), (((7, 0, math.inf), (3, 0, 1)), 9014),
