@@ -229,7 +229,7 @@ void oracle_cluster(const uint16_t *q, const uint16_t *k, int n, int d, int Cq, 
 }
 
 /* Cluster-pair importance ([PSA] sec. 2 on SVG2: centroid-level scores     */
-/* and top-k cluster selection; [iCATS] 4 "cluster-level scores").           */
+/* and top-k cluster selection; [iCATS] 4, scores at the cluster level).     */
 /* Reading: importance = estimated attention mass of the pair. Query cluster */
 /* a puts softmax weight n_b e^{s_ab} / Z_a on key cluster b, with           */
 /*   s_ab = scale * mu_a . c_b,  Z_a = sum_b n_b e^{s_ab - m_a},             */
