@@ -511,6 +511,55 @@ def run_gpu(args):
     return 0
 
 
+def run_cluster_report(args):
+    """Clustering stage alone at the Wan2.1-14B call, three ways (one JSON line,
+    not the benchmark line): the cold 10-round co-clustering the bench step
+    runs, the same with the identity metric (independent k-means of each side),
+    and a 2-round warm start from the cold result (the next timestep's call)."""
+    import dataclasses
+    import torch
+
+    import free_sparse_attention_head_b200 as svoo
+    from free_sparse_attention_head_b200 import build as svoo_build
+
+    svoo_build.build()
+    svoo.load()
+    dev = torch.device("cuda", 0)
+    w = workload.get(WORKLOAD)
+    if args.heads:
+        w = dataclasses.replace(w, H=args.heads)
+    q, k, _ = workload.make_qkv(w)
+    as_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16).view(w.B, w.H, w.N, w.d)
+    qd, kd = as_dev(q), as_dev(k)
+    del q, k
+    sh = svoo.make_shape(qd)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    base = svoo.Config(n_qc=w.n_qc, n_kc=w.n_kc, iters=w.iters, block_q=w.block_q)
+    ws = torch.empty(svoo.workspace_sizes(sh, base)[0], dtype=torch.uint8, device=dev)
+    cold = svoo.cluster(qd, kd, base, workspace=ws, dev_err=err)
+    warm_state = (cold["q_cent"], cold["k_cent"], cold["k_sizes"])
+    cases = {
+        "cold_interaction_10": (base, None),
+        "cold_identity_10": (dataclasses.replace(base, metric=1), None),
+        "warm_interaction_2": (dataclasses.replace(base, iters=2), warm_state),
+    }
+    res = {}
+    for name, (cfg, warm) in cases.items():
+        for _ in range(max(args.warmup, 3)):
+            svoo.cluster(qd, kd, cfg, warm=warm, workspace=ws, dev_err=err)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            svoo.cluster(qd, kd, cfg, warm=warm, workspace=ws, dev_err=err)
+        e1.record()
+        torch.cuda.synchronize()
+        svoo.check_device_errors(err)
+        res[name] = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"report": "clustering stage, ms per call", "workload": f"{w.name}, H={w.H}, N={w.N}",
+                      "steps": args.steps, "warmup": args.warmup, "ms": res}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -522,7 +571,11 @@ def main():
                     help="plan source: online co-clustering (default) or PSA's static stripe mask")
     ap.add_argument("--heads", type=int, default=0,
                     help="run the first H heads only (smaller profiling captures; not a bench line)")
+    ap.add_argument("--cluster-report", action="store_true",
+                    help="time the clustering stage alone (cold, identity metric, warm start); not a bench line")
     args = ap.parse_args()
+    if args.cluster_report:
+        return run_cluster_report(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)
