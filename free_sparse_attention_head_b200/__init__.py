@@ -25,7 +25,7 @@ __all__ = [
     "Config", "Shape", "Plan", "load", "lib_path", "cluster", "cluster_step", "build_mask",
     "permute", "sparse_attn", "sparse_attention", "check_device_errors", "workspace_sizes",
     "SvooError", "CLUSTER_WARM", "CLUSTER_IDENTITY", "PSA_INF", "psa_config", "psa_params",
-    "psa_mask", "psa_attention",
+    "psa_mask", "psa_attention", "snr_top_p", "cluster_outputs",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +72,7 @@ _SIGS = {
     "svoo_sparse_attn": (_I, [_SP, _P, _P, _P, _PP, _I, _I, _I, _F, _P, _P, _P]),
     "svoo_psa_block_count": (_I, [_I, _I, _I, _I, _I, _I]),
     "svoo_psa_mask": (_I, [_SP, _I, _I, _I, _I, _I, _I, _P, _I, _PP, _P, _P, _P]),
+    "svoo_snr_top_p": (_I, [_I, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double, _P]),
 }
 
 EXPORTS = tuple(_SIGS)
@@ -236,26 +237,46 @@ def _cluster_flags(cfg: Config, warm) -> int:
     return (CLUSTER_WARM if warm is not None else 0) | (CLUSTER_IDENTITY if cfg.metric == 1 else 0)
 
 
-def cluster(q, k, cfg: Config, n_text=0, warm=None, workspace=None, dev_err=None, stream=None):
-    """Co-clusters the video tokens of every head; returns a dict of device tensors."""
+_CLUSTER_OUT = ("q_assign", "k_assign", "q_cent", "k_cent", "q_sizes", "k_sizes")
+
+
+def cluster_outputs(shape: Shape, cfg: Config, device) -> dict:
+    """Device output buffers of `cluster` for a shape, to be reused across calls."""
+    BH, nv, d = shape.B * shape.H, shape.N - shape.n_text, shape.d
+    return dict(
+        q_assign=torch.empty(BH, nv, dtype=torch.int32, device=device),
+        k_assign=torch.empty(BH, nv, dtype=torch.int32, device=device),
+        q_cent=torch.empty(BH, cfg.n_qc, d, dtype=torch.float32, device=device),
+        k_cent=torch.empty(BH, cfg.n_kc, d, dtype=torch.float32, device=device),
+        q_sizes=torch.zeros(BH, cfg.n_qc, dtype=torch.int32, device=device),
+        k_sizes=torch.zeros(BH, cfg.n_kc, dtype=torch.int32, device=device),
+    )
+
+
+def cluster(q, k, cfg: Config, n_text=0, warm=None, workspace=None, dev_err=None, stream=None,
+            out: Optional[dict] = None):
+    """Co-clusters the video tokens of every head; returns a dict of device tensors.
+
+    `out` (from cluster_outputs) is written in place instead of allocating new
+    outputs. warm = (q_cent, k_cent, k_sizes) starts from those centroids
+    (SVOO_CLUSTER_WARM); they may be out's own tensors (the previous call's
+    result), in which case nothing is copied."""
     _need_cuda(q, k)
     sh = make_shape(q, n_text)
-    BH, nv, d = sh.B * sh.H, sh.N - n_text, sh.d
     dev = q.device
     if workspace is None:
         workspace = torch.empty(workspace_sizes(sh, cfg)[0], dtype=torch.uint8, device=dev)
-    out = dict(
-        q_assign=torch.empty(BH, nv, dtype=torch.int32, device=dev),
-        k_assign=torch.empty(BH, nv, dtype=torch.int32, device=dev),
-        q_cent=torch.empty(BH, cfg.n_qc, d, dtype=torch.float32, device=dev),
-        k_cent=torch.empty(BH, cfg.n_kc, d, dtype=torch.float32, device=dev),
-        q_sizes=torch.zeros(BH, cfg.n_qc, dtype=torch.int32, device=dev),
-        k_sizes=torch.zeros(BH, cfg.n_kc, dtype=torch.int32, device=dev),
-    )
+    if out is None:
+        out = cluster_outputs(sh, cfg, dev)
+    else:
+        missing = [f for f in _CLUSTER_OUT if f not in out]
+        if missing:
+            raise SvooError(f"cluster(out=...) lacks {missing}")
+        _need_cuda(*(out[f] for f in _CLUSTER_OUT))
     if warm is not None:
-        out["q_cent"].copy_(warm[0])
-        out["k_cent"].copy_(warm[1])
-        out["k_sizes"].copy_(warm[2])
+        for dst, src in zip(("q_cent", "k_cent", "k_sizes"), warm):
+            if out[dst].data_ptr() != src.data_ptr():
+                out[dst].copy_(src)
     err = _err_buf(dev_err, dev)
     _check(load().svoo_cluster(ctypes.byref(sh), _ptr(q), _ptr(k), cfg.n_qc, cfg.n_kc, cfg.iters,
                                _cluster_flags(cfg, warm), _ptr(out["q_assign"]), _ptr(out["k_assign"]),
@@ -411,3 +432,17 @@ def psa_attention(q, k, v, grid, block, params: torch.Tensor, n_text=0, block_q:
     qp, kp, vp = permute(q, k, v, k_assign, plan, dev_err=err, stream=stream)
     out = sparse_attn(qp, kp, vp, plan, dev_err=err, stream=stream)
     return out, dict(plan=plan, k_assign=k_assign, dev_err=err, cfg=cfg)
+
+
+# --------------------------------------------------------------------------- SNR-guided top-p
+
+
+def snr_top_p(steps: int, warmup: int = 0, p_min: float = 0.7, tau: float = 0.999,
+              shift: float = 1.0):
+    """Top-p of each of `steps` denoising calls (svoo_snr_top_p), as a float32
+    numpy array; feed p[t] to build_mask with Config(select_mode=1)."""
+    import numpy as np
+    p = np.empty(int(steps), dtype=np.float32)
+    _check(load().svoo_snr_top_p(int(steps), int(warmup), float(p_min), float(tau), float(shift),
+                                 p.ctypes.data_as(ctypes.c_void_p)), "svoo_snr_top_p")
+    return p

@@ -17,9 +17,9 @@
 //   warps 4-7   softmax of tile A, warps 8-11 softmax of tile B: thread r owns
 //               query row r (= TMEM lane r); reads S_t(j), masks invalid keys,
 //               keeps the running max (rescaling O_t in TMEM only when the max
-//               grows by more than 2^8) and sum, writes P_t(j) as packed bf16
-//               into the upper half of S_t's columns, from where the next MMA
-//               reads it as its A operand
+//               grows by more than 2^8) and the sum of the bf16-rounded P,
+//               writes P_t(j) as packed bf16 into the upper half of S_t's
+//               columns, from where the next MMA reads it as its A operand
 //   warps 2-3   idle
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+d), O_B [384,384+d).
 // The producer / consumer split follows the flash-attention pipeline that the
@@ -66,6 +66,20 @@ __device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// acc + lo + hi of a packed bf16 pair, each widened exactly and added in fp32
+// (sm_100 mixed-precision add): the row sum sees the same rounded P that the
+// PV product consumes, so the normalisation matches the numerator.
+__device__ __forceinline__ float add_bf16x2(uint32_t pk, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {lo, hi}, %1;\n\t"
+      "add.rn.f32.bf16 t, lo, %2;\n\t"
+      "add.rn.f32.bf16 %0, hi, t;\n\t}"
+      : "=f"(r)
+      : "r"(pk), "f"(acc));
+  return r;
 }
 
 // Walks the chunk sequence in increasing order: group of chunk gc, its first
@@ -348,7 +362,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float neg_m = -m;
       // P = 2^(s scale_log2 - m), packed bf16 pairs into the upper half of S_t's
       // columns; the first 64 keys are released to the MMA before the rest
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
@@ -356,8 +370,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < 16; ++c) {
           const float p0 = ex2_approx(fmaf(s[q * 32 + 2 * c], scale_log2, neg_m));
           const float p1 = ex2_approx(fmaf(s[q * 32 + 2 * c + 1], scale_log2, neg_m));
-          rs4[c & 3] += p0 + p1;
           pk[c] = pack_bf16x2(p0, p1);
+          rs8[c & 7] = add_bf16x2(pk[c], rs8[c & 7]);
         }
         tmem_st16(lane_base + s_col + kPOff + q * 16, pk);
         if (q == 1) {
@@ -381,7 +395,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (lane == 0) mbar_arrive(smem_u32(&S->p_half[t]));
         }
       }
-      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
       l = l * alpha + rs;
       tmem_wait_st();
       tc_fence_before();

@@ -1043,6 +1043,12 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
 
 bool cluster_counts_ok(int C) { return C >= 1 && C <= 256; }
 
+// Cluster count that sizes a half-step's scratch: metric_C only counts when a
+// metric is given (it is ignored, whatever its value, for the identity).
+int step_clusters(int C, const float* metric_cent, int metric_C) {
+  return (metric_cent && metric_C > C) ? metric_C : C;
+}
+
 }  // namespace
 }  // namespace svoo
 
@@ -1063,7 +1069,7 @@ extern "C" svoo_status svoo_cluster_step(const svoo_shape* shape, const void* x,
   if (!aligned(x, 16)) return SVOO_ERR_INVALID_ARG;
   const int BH = bh_of(shape);
   StepWs w;
-  size_t need = carve_step(workspace, BH, shape->d, C > metric_C ? C : metric_C, &w);
+  size_t need = carve_step(workspace, BH, shape->d, step_clusters(C, metric_cent, metric_C), &w);
   if (workspace_bytes < need) return SVOO_ERR_WORKSPACE;
   return run_step(shape, x, C, cent, sizes, assign, metric_cent, metric_sizes, metric_C, w, dev_err,
                   static_cast<cudaStream_t>(stream), C);
@@ -1160,7 +1166,7 @@ extern "C" svoo_status svoo_cluster_step_static(const svoo_shape* shape, const v
   if (metric_cent && (!metric_sizes || !cluster_counts_ok(metric_C))) return SVOO_ERR_INVALID_ARG;
   if (!aligned(x, 16)) return SVOO_ERR_INVALID_ARG;
   const int BH = bh_of(shape);
-  const int Cmax = C > metric_C ? C : metric_C;
+  const int Cmax = step_clusters(C, metric_cent, metric_C);
   if (carve_step(nullptr, BH, shape->d, Cmax, nullptr) > kStaticScratchBytes)
     return SVOO_ERR_WORKSPACE;  // shape needs more than the fixed scratch holds
   int dev = 0;

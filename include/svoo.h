@@ -157,8 +157,9 @@ svoo_status svoo_cluster(const svoo_shape *shape, const void *q, const void *k, 
 
 /* One half-step of the above for one side: assigns the video tokens of x to
  * the centroids `cent` (in/out) under the metric of (metric_cent, metric_sizes)
- * (metric_C clusters; identity if metric_cent is NULL), then updates `cent`
- * and `sizes`. Used for warm starts and for step-level parity checks. */
+ * (metric_C clusters; identity if metric_cent is NULL, and metric_C is then
+ * ignored), then updates `cent` and `sizes`. Used for warm starts and for
+ * step-level parity checks. */
 svoo_status svoo_cluster_step(const svoo_shape *shape, const void *x, int C, float *cent,
                               int32_t *sizes, int32_t *assign, const float *metric_cent,
                               const int32_t *metric_sizes, int metric_C, void *workspace,
@@ -270,6 +271,23 @@ svoo_status svoo_permute(const svoo_shape *shape, const void *q, const void *k, 
 svoo_status svoo_sparse_attn(const svoo_shape *shape, const void *qp, const void *kp,
                              const void *vp, const svoo_plan *plan, int n_qc, int n_kc,
                              int block_q, float scale, void *o, int32_t *dev_err, void *stream);
+
+/* ------------------------------------------------------------------ top-p schedule
+ * SNR-guided top-p of every call of a denoising run ("iCATS" section 4.2 and
+ * appendix A: top-p follows a smooth function of the log signal-to-noise
+ * ratio, fixed offline from the noise schedule, with dense attention before
+ * the first sparse call; the budget stays steady early and late and falls in
+ * the middle). The pages give no formula; this library reads it as
+ *   s = 1 - t/steps, sigma = shift*s / (1 + (shift - 1)*s)   (flow matching),
+ *   p(t) = p_min + (tau - p_min) / (1 + SNR(t)),  SNR = ((1 - sigma)/sigma)^2,
+ * i.e. a logistic in log SNR: tau at pure noise, p_min in the noise-free
+ * limit, (tau + p_min)/2 where SNR = 1; p(t) = 1 for t < warmup.
+ * Host code only (no GPU work): writes p[0..steps-1] (HOST memory, fp32),
+ * ready to be passed as the per-head keep values of svoo_build_mask with
+ * select_mode 1. Requires steps >= 1, warmup >= 0, 0 <= p_min <= tau <= 1,
+ * shift > 0; otherwise SVOO_ERR_INVALID_ARG and p is left untouched. */
+svoo_status svoo_snr_top_p(int steps, int warmup, double p_min, double tau, double shift,
+                           float *p);
 
 const char *svoo_status_string(svoo_status s);
 

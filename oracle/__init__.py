@@ -62,6 +62,7 @@ _SIGS = {
     "oracle_dense_attn_rows": (None, [_P, _P, _P, _I, _I, _F, _P, _I, _P]),
     "oracle_psa_attends": (_I, [ctypes.c_longlong, ctypes.c_longlong, ctypes.c_longlong, _P]),
     "oracle_psa_plan": (_I, [_I, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
+    "oracle_snr_top_p": (_I, [_I, _I, ctypes.c_double, ctypes.c_double, ctypes.c_double, _P]),
 }
 
 
@@ -320,3 +321,13 @@ def psa_plan_head(T, H, W, block, n_text, prm, block_q):
     return dict(kmask=p["kmask"], q_label=p["label"], k_label=p["label"], q_sizes=p["sizes"],
                 nb=p["nb"], q_perm=q_perm, q_off=q_off, k_perm=q_perm, k_off=q_off,
                 tiles=tiles(q_off, block_q))
+
+
+# --------------------------------------------------------------------------- SNR-guided top-p
+
+def snr_top_p(steps, warmup=0, p_min=0.7, tau=0.999, shift=1.0):
+    """Top-p of each of `steps` denoising calls (fp32 [steps]); see oracle_snr_top_p."""
+    p = np.empty(steps, dtype=np.float32)
+    if lib().oracle_snr_top_p(int(steps), int(warmup), float(p_min), float(tau), float(shift), _p(p)) != 0:
+        raise ValueError("bad SNR schedule arguments")
+    return p

@@ -633,3 +633,41 @@ int oracle_psa_plan(int T, int H, int W, int bt, int bh, int bw, int n_text, con
     }
     return nb;
 }
+
+/* ------------------------------------------------------------------------ */
+/* [iCATS] 4.2 and appendix A: the top-p of each denoising call follows a     */
+/* smooth function of log SNR, fixed offline from the noise schedule; calls   */
+/* before the first sparse one stay dense; the budget is steady early and     */
+/* late and falls in the middle; tau and p_min are its parameters. The pages  */
+/* give no formula. Reading (parity unpinned by the pages):                   */
+/*   noise level of call t (flow matching, t = 0 is pure noise, `shift` the   */
+/*   usual timestep shift):  s = 1 - t/steps,  sigma = shift s / (1 + (shift-1) s) */
+/*   lambda = log SNR = 2 ln((1 - sigma) / sigma)                             */
+/*   p(t) = p_min + (tau - p_min) / (1 + e^lambda)   for t >= warmup,         */
+/*   p(t) = 1                                        for t <  warmup.         */
+/* So p = tau at pure noise, p_min in the noise-free limit, and the midpoint  */
+/* (tau + p_min) / 2 where SNR = 1; the logistic in lambda keeps both ends    */
+/* flat. The value is rounded once to fp32 (build_mask takes an fp32 p).      */
+/* ------------------------------------------------------------------------ */
+int oracle_snr_top_p(int steps, int warmup, double p_min, double tau, double shift, float *p) {
+    if (steps < 1 || warmup < 0 || !(p_min >= 0.0) || !(tau >= p_min) || !(tau <= 1.0) ||
+        !(shift > 0.0) || !p)
+        return -1;
+    for (int t = 0; t < steps; ++t) {
+        if (t < warmup) {
+            p[t] = 1.0f;
+            continue;
+        }
+        double s = 1.0 - (double)t / (double)steps;
+        double sigma = shift * s / (1.0 + (shift - 1.0) * s);
+        double noisy_share;
+        if (sigma >= 1.0) {
+            noisy_share = 1.0; /* lambda = -infinity */
+        } else {
+            double lambda = 2.0 * log((1.0 - sigma) / sigma);
+            noisy_share = 1.0 / (1.0 + exp(lambda));
+        }
+        p[t] = (float)(p_min + (tau - p_min) * noisy_share);
+    }
+    return 0;
+}

@@ -99,6 +99,11 @@ int oracle_psa_attends(long long i, long long j, long long HW, const int32_t *pr
 int oracle_psa_plan(int T, int H, int W, int bt, int bh, int bw, int n_text, const int32_t *prm,
                     int32_t *label, uint64_t *kmask, int32_t *sizes);
 
+/* [iCATS] 4.2, appendix A: SNR-guided top-p of each of `steps` denoising
+ * calls (a reading: the pages give the shape of the schedule, not a formula;
+ * see the .c file). Writes p[0..steps-1]; returns 0, or -1 for bad arguments. */
+int oracle_snr_top_p(int steps, int warmup, double p_min, double tau, double shift, float *p);
+
 #ifdef __cplusplus
 }
 #endif

@@ -141,3 +141,24 @@ def test_psa_block_count_and_mask_validation(lib):
     assert lib.svoo_psa_mask(*args(ok, pl=None)) == 1
     empty = svoo._CPlan(*([0] * 12))
     assert lib.svoo_psa_mask(*args(ok, pl=ctypes.byref(empty))) == 1
+
+
+@pytest.mark.parametrize("args", [(50, 0, 0.7, 0.999, 1.0), (50, 5, 0.7, 0.999, 5.0),
+                                  (30, 2, 0.5, 0.95, 3.0), (7, 0, 0.8, 0.8, 1.0)])
+def test_snr_top_p_schedule_matches_oracle(lib, args):
+    """svoo_snr_top_p is host code (no device work): the library's schedule
+    equals the oracle's, written separately from the same reading of iCATS
+    section 4.2, to one fp32 rounding."""
+    import numpy as np
+    import oracle
+    got = svoo.snr_top_p(*args).astype(np.float64)
+    want = oracle.snr_top_p(*args).astype(np.float64)
+    assert np.all(np.abs(got - want) <= np.spacing(np.float32(1.0)))
+
+
+def test_snr_top_p_rejects_bad_arguments(lib):
+    for bad in [(0, 0, 0.7, 0.9, 1.0), (10, -1, 0.7, 0.9, 1.0), (10, 0, 0.9, 0.7, 1.0),
+                (10, 0, 0.7, 1.5, 1.0), (10, 0, 0.7, 0.9, -2.0)]:
+        with pytest.raises(svoo.SvooError):
+            svoo.snr_top_p(*bad)
+    assert lib.svoo_snr_top_p(5, 0, 0.7, 0.9, 1.0, None) == 1

@@ -516,3 +516,57 @@ def test_generator_deterministic_and_subsettable():
     assert abs(f.std() - math.sqrt(4 + 0.25)) < 0.5
     assert f32_to_bf16_bits(np.array([1.0 + 2 ** -8], np.float32))[0] == 0x3F80  # tie to even
     assert f32_to_bf16_bits(np.array([1.0 + 3 * 2 ** -8], np.float32))[0] == 0x3F82
+
+
+# ----------------------------------------------------------------------------- SNR-guided top-p
+# iCATS section 4.2 / appendix A give the shape of the schedule only (dense
+# before the first sparse call, steady early and late, falling in the middle,
+# a smooth function of log SNR, parameters tau and p_min); the formula is a
+# reading, so these pins check the stated properties and the closed-form
+# points of that reading, not values printed on the pages (parity unpinned).
+
+
+def test_snr_schedule_warmup_dense_and_starts_at_tau():
+    p = oracle.snr_top_p(50, warmup=4, p_min=0.7, tau=0.999)
+    assert (p[:4] == 1.0).all()
+    q = oracle.snr_top_p(50, warmup=0, p_min=0.7, tau=0.999)
+    assert q[0] == np.float32(0.999)          # pure noise: SNR = 0
+    assert np.array_equal(p[4:], q[4:])         # warm-up does not shift the schedule
+
+
+@pytest.mark.parametrize("shift", [1.0, 3.0, 5.0])
+def test_snr_schedule_monotone_between_p_min_and_tau(shift):
+    p = oracle.snr_top_p(200, warmup=0, p_min=0.6, tau=0.99, shift=shift).astype(np.float64)
+    assert (np.diff(p) <= 0).all()
+    assert p.min() > 0.6 - 1e-7 and p.max() <= 0.99 + 1e-7
+    # noise-free limit: the last of many steps is close to p_min
+    assert oracle.snr_top_p(100000, 0, 0.6, 0.99, shift)[-1] < 0.6 + 1e-6
+
+
+@pytest.mark.parametrize("steps,shift,t_mid", [(50, 1.0, 25), (40, 3.0, 30), (60, 5.0, 50)])
+def test_snr_schedule_midpoint_where_snr_is_one(steps, shift, t_mid):
+    """SNR = 1 where the shifted noise level is 1/2, i.e. s = 1 / (1 + shift),
+    t = steps (1 - s): there p is the mean of tau and p_min."""
+    p = oracle.snr_top_p(steps, 0, 0.7, 0.999, shift)
+    assert abs(float(p[t_mid]) - (0.7 + 0.999) / 2) < 1e-7
+    assert p[t_mid - 1] > p[t_mid] > p[t_mid + 1]
+
+
+def test_snr_schedule_is_logistic_in_log_snr():
+    """Equal steps in log SNR away from SNR = 1 give mirror-image distances
+    from the midpoint (the logistic's odd symmetry)."""
+    steps = 1000
+    p = oracle.snr_top_p(steps, 0, 0.5, 0.9).astype(np.float64)
+    sigma = 1.0 - np.arange(steps) / steps
+    lam = 2.0 * np.log((1.0 - sigma[1:]) / sigma[1:])
+    for a, b in [(100, 900), (250, 750), (400, 600)]:   # lambda(b) = -lambda(a)
+        assert abs(lam[a - 1] + lam[b - 1]) < 1e-9
+        assert abs((p[a] - 0.7) + (p[b] - 0.7)) < 1e-6
+
+
+def test_snr_schedule_flat_when_tau_equals_p_min_and_rejects_bad_args():
+    assert (oracle.snr_top_p(30, 0, 0.8, 0.8) == np.float32(0.8)).all()
+    for bad in [(0, 0, 0.7, 0.9, 1.0), (10, -1, 0.7, 0.9, 1.0), (10, 0, 0.9, 0.7, 1.0),
+                (10, 0, 0.7, 1.5, 1.0), (10, 0, 0.7, 0.9, 0.0), (10, 0, -0.1, 0.9, 1.0)]:
+        with pytest.raises(ValueError):
+            oracle.snr_top_p(*bad)

@@ -104,3 +104,41 @@ def test_static_scratch_rejects_oversized_shape():
     st = lib.svoo_cluster_step_static(ctypes.byref(sh), fake, 256, fake, fake, fake, None, None, 0,
                                       None, None)
     assert st == 2 and lib.svoo_status_string(st) == b"workspace too small"
+
+
+def test_static_scratch_ignores_metric_count_without_metric():
+    """With no metric (identity), metric_C plays no part: 40 heads, d = 128 and
+    128 clusters fit the fixed scratch while 256 would not, so a leftover
+    metric_C = 256 beside a NULL metric must neither be refused nor change the
+    result (same labels and sizes as the workspace entry point)."""
+    svoo_build.build()
+    lib = svoo.load()
+    B, H, N, d, C = 1, 40, 1024, 128, 128
+    rng = np.random.Generator(np.random.PCG64(5))
+    x = workload.f32_to_bf16_bits(rng.standard_normal((B * H, N, d), dtype=np.float32))
+    xd = _dev_bf16(x, B, H)
+    c0 = _token_start(x, C)
+    res = []
+    for static in (False, True):
+        cent = torch.from_numpy(c0.copy()).cuda()
+        sizes = torch.zeros(B * H, C, dtype=torch.int32, device="cuda")
+        assign = torch.full((B * H, N), -1, dtype=torch.int32, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sh = svoo.Shape(B, H, N, d, 0)
+        P = lambda t: ctypes.c_void_p(t.data_ptr())
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        if static:
+            st = lib.svoo_cluster_step_static(ctypes.byref(sh), P(xd), C, P(cent), P(sizes), P(assign),
+                                              None, None, 256, P(err), stream)
+        else:
+            ws_bytes = lib.svoo_cluster_workspace_size(ctypes.byref(sh), C, C)
+            ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+            st = lib.svoo_cluster_step(ctypes.byref(sh), P(xd), C, P(cent), P(sizes), P(assign), None,
+                                       None, 256, P(ws), ws_bytes, P(err), stream)
+        assert st == 0, lib.svoo_status_string(st)
+        torch.cuda.synchronize()
+        svoo.check_device_errors(err)
+        res.append((assign, sizes))
+    assert torch.equal(res[0][0], res[1][0])
+    assert torch.equal(res[0][1], res[1][1])
+    assert int(res[1][1].sum()) == B * H * N

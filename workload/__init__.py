@@ -35,7 +35,7 @@ import numpy as np
 __all__ = [
     "Workload", "WORKLOADS", "get", "splitmix64", "f32_to_bf16_bits",
     "bf16_bits_to_f32", "make_qkv", "cell_centers", "sweep_workload", "psa_strategies",
-    "PSA_BLOCKS",
+    "PSA_BLOCKS", "next_timestep",
 ]
 
 _MASK64 = np.uint64(0xFFFFFFFFFFFFFFFF)
@@ -176,6 +176,16 @@ def make_qkv(w: Workload, heads: Optional[Sequence[int]] = None):
             k[i, nv:] = f32_to_bf16_bits(np.float32(2.0) * rng.standard_normal((nt, d), dtype=np.float32))
             v[i, nv:] = f32_to_bf16_bits(rng.standard_normal((nt, d), dtype=np.float32))
     return q, k, v
+
+
+def next_timestep(x: np.ndarray, sigma: float = 0.1, seed: int = 1) -> np.ndarray:
+    """Inputs of the next denoising call, standing in for the slow drift of a
+    layer's Q or K from one timestep to the next: x + sigma N(0, I) per token,
+    drawn from PCG64(seed) as float32 and rounded to bf16 (uint16 bits, same
+    shape as x)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    noise = rng.standard_normal(x.shape, dtype=np.float32)
+    return f32_to_bf16_bits(bf16_bits_to_f32(x) + np.float32(sigma) * noise)
 
 
 WORKLOADS = {
