@@ -40,6 +40,10 @@ constexpr int kTmemS0 = 0;     // S_A; S_B at +128
 constexpr int kTmemO0 = 256;   // O_A; O_B at +128
 constexpr int kPOff = 64;      // P_t within S_t's columns (64 packed bf16 pairs)
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kRegsLaunch = 168;  // 65536 / 384, rounded down to a multiple of 8
+constexpr int kRegsLow = 64;      // warps 0-3: TMA producer, MMA issuer
+constexpr int kRegsHigh = 216;    // warps 4-11: softmax of the two query tiles
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kAttnThreads * kRegsLaunch, "register split");
 
 struct AttnSmem {
   uint64_t q_full;
@@ -206,6 +210,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int oob_row = BH * N;  // past the tensor: TMA fills zeros
   const uint32_t q_u = smem_u32(q_s), k_u = smem_u32(k_s), v_u = smem_u32(v_s);
 
+  // registers: the producer / issuer warpgroup gives up what the softmax
+  // warpgroups use (launch: 384 x 168 = 128 x kRegsLow + 256 x kRegsHigh);
+  // each warpgroup's branch starts with its own setmaxnreg
+  if (warp < 4) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0 && nkv > 0) {
     // ---------------------------------------------------------------- producer
     int k_armed = -1, v_armed = -1;  // last tile whose K / V load was issued
@@ -307,7 +316,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int dummy = 0;
       mbar_wait(smem_u32(&S->mma_final), 0, &dummy);
     }
-  } else if (warp >= 4 && (warp < 8 || has_b)) {
+  }
+  } else {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+  if (warp < 8 || has_b) {
     // ---------------------------------------------------------------- softmax of tile t
     const int t = (warp - 4) >> 2;
     const int r = tid - 128 * (1 + t);  // query row within the tile == TMEM lane
@@ -347,29 +359,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int c = 0; c < kChunkRows; ++c)
             if (c >= vmask[c8]) s[c8 * kChunkRows + c] = -INFINITY;
       }
-      // row max (raw scores; scale_log2 > 0 keeps the order), 8 independent chains
-      float m8[8];
+      // row max (raw scores; scale_log2 > 0 keeps the order): four chains of
+      // three-input maxima
+      float m4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) m8[e] = s[e];
-#pragma unroll
-      for (int c = 8; c < kKvRows; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * scale_log2;
+      for (int c = 4; c < kKvRows; c += 8) {
+        m4[0] = fmax3(m4[0], s[c], s[c + 1]);
+        m4[1] = fmax3(m4[1], s[c + 2], s[c + 3]);
+        if (c + 4 < kKvRows) {
+          m4[2] = fmax3(m4[2], s[c + 4], s[c + 5]);
+          m4[3] = fmax3(m4[3], s[c + 6], s[c + 7]);
+        }
+      }
+      const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * scale_log2;
       // running max (log2 units): moved only when it grows by more than 2^8 (P stays <= 2^8)
       const bool grow = mx > m + kRescaleLog2;
       const float alpha = (j > 0 && grow) ? ex2_approx(m - mx) : 1.f;
       if (grow || j == 0) m = fmaxf(m, mx);
-      const float neg_m = -m;
-      // P = 2^(s scale_log2 - m), packed bf16 pairs into the upper half of S_t's
-      // columns; the first 64 keys are released to the MMA before the rest
+      // P = 2^(s scale_log2 - m) (argument by packed fp32 pairs), packed bf16
+      // pairs into the upper half of S_t's columns; the first 64 keys are
+      // released to the MMA before the rest
+      const uint64_t sc2 = f2pack(scale_log2, scale_log2), nm2 = f2pack(-m, -m);
       float rs8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2_approx(fmaf(s[q * 32 + 2 * c], scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(s[q * 32 + 2 * c + 1], scale_log2, neg_m));
+          float x0, x1, p0, p1;
+          f2unpack(f2fma(f2pack(s[q * 32 + 2 * c], s[q * 32 + 2 * c + 1]), sc2, nm2), x0, x1);
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
           pk[c] = pack_bf16x2(p0, p1);
           rs8[c & 7] = add_bf16x2(pk[c], rs8[c & 7]);
         }
@@ -435,6 +455,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < D / 8; ++c) orow[c] = make_uint4(0, 0, 0, 0);
       }
     }
+  }
   }
   tc_fence_before();
   __syncthreads();
