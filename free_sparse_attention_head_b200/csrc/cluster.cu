@@ -8,13 +8,15 @@
 //   metric_m_kernel   M from the other side's centroids and sizes (fp64)
 //   metric_nu_kernel  nu_j = M mu_j, kappa_j = mu_j . nu_j (fp64), |nu_j|, and
 //                     nu_j split into two bf16 rows (hi + lo)
-//   assign_kernel     persistent, warp-specialised: tcgen05 MMAs of 128-token
-//                     tiles against [nu_hi | nu_lo] into double-buffered TMEM;
-//                     per token the score kappa_j - 2 x.nu_j is bounded by the
-//                     MMA error, a token with a single candidate takes it and
-//                     the rest are re-scored in fp64 (ties to the smaller j);
-//                     member sums in fp64 (exact, so order-independent) and
-//                     counts, added atomically.
+//   assign_kernel     persistent, warp-specialised, dynamically scheduled:
+//                     tcgen05 MMAs of 128-token tiles against [nu_hi | nu_lo]
+//                     into double-buffered TMEM; per token the score
+//                     kappa_j - 2 x.nu_j is bounded by the MMA error and a
+//                     token with a single candidate takes it
+//   fixup_kernel      the other tokens: candidates re-scored closer, then in
+//                     fp64 (ties to the smaller j)
+//   update_kernel     member sums in fp64, exact (so order-independent), per
+//                     chunk of consecutive tokens grouped by label
 //   finalize_kernel   centroid = fp32(sum / count), empty clusters keep
 //                     theirs; resets the sums for the next half-step.
 #include <math.h>
@@ -281,29 +283,33 @@ __global__ void __launch_bounds__(128)
 }
 inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d) * sizeof(double); }
 
-// ---------------------------------------------------------------- assign + update
+// ---------------------------------------------------------------- assign
 //
-// Persistent, warp-specialised kernel, one CTA per SM, each CTA walking a
-// contiguous stretch of the (head, 128-token tile) sequence. Tile i uses X
-// buffer i % 2 in shared memory and TMEM accumulator i % 2 (CP fp32 columns).
+// Persistent, warp-specialised kernel, one CTA per SM. The (head, 128-token
+// tile) space is handed out in chunks of kChunkTiles tiles of one head through
+// per-head counters: a CTA starts at its own head and moves on to the next
+// head with chunks left, so SMs that run this kernel faster take more chunks
+// (on B200 some SMs ran the same tiles up to 1.5x slower than others, so a
+// static split left the fast ones idle). Tile i of a CTA uses X buffer i % 2
+// in shared memory and TMEM accumulator i % 2 (CP fp32 columns).
 //   producer (warp 0)   TMA of the X tile, then one tcgen05 chain per tile:
 //                       u = X . nu_hi^T + X . nu_lo^T + 1 . (-kappa/2)^T, the
 //                       last term a 16-wide K chunk of ones against -kappa_j/2
 //                       split into three bf16 parts, so u_j = x.nu_j - kappa_j/2
 //                       and the score is kappa_j - 2 x.nu_j = -2 u_j.
-//   scorers (warps 8-15) thread (row r, column half): |x|^2 over half of the
-//                       dimensions (then the X buffer goes back), the half's
-//                       maximum of u, and, with the row maximum U and the error
-//                       bound E, its candidates u_j >= U - 2E (they contain the
-//                       exact argmin of the score; then the accumulator goes
-//                       back). A row with one candidate takes it; the others
-//                       are deferred with their candidate list.
-//   summers (warps 1-7) warp w owns rows [128(w-1)/7, 128w/7) of every tile:
-//                       member sums of the labelled rows (re-read from L2), a
-//                       run of equal labels in token order summed in fp32 and
-//                       added with one vector atomic per lane, and the deferred
-//                       rows, decided from the shared-memory nu copies or, inside
-//                       that bound, by an fp64 re-score (ties to the smaller j).
+//   scorers (warps 1-16) warp w reads TMEM lane quarter w % 4 (32 rows) and
+//                       column quarter (w - 1) / 4: each thread loads its row's
+//                       CP/4 scores into registers (then the accumulator goes
+//                       back), the quarter's maximum; the four quarters of a
+//                       row meet in shared memory for the row maximum U and
+//                       the error bound E; then each thread lists its
+//                       quarter's candidates u_j >= U - 2E (they contain the
+//                       exact argmin of the score). The quarter-0 warp of a
+//                       lane quarter decides its rows: one candidate is the
+//                       label; several go to the tile's deferred list (up to
+//                       kDeferSlots rows per 32 with up to kDeferCand
+//                       candidates each, label -1) or, beyond that, get label
+//                       -2 (all clusters); fixup_kernel decides them.
 //
 // Error bound: nu_hi + nu_lo equals nu to 2^-18 relative and the three kappa
 // parts give kappa to 2^-26; the MMA's fp32 accumulation of 2d + 3 exact
@@ -311,37 +317,44 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 // |x||nu_j| (1 + 2^-8) + |kappa_j| / 2. E = 2^-13 (|x| max|nu| + max|kappa| / 2)
 // bounds |u_computed - u| with a factor of two to spare.
 
-constexpr int kScorerWarps = 8;
-constexpr int kSummerWarps = 7;
-// warp 0 is the producer; the summers take the next warp ids, the scorers the last
-constexpr int kFirstSummer = 1;
-constexpr int kFirstScorer = kFirstSummer + kSummerWarps;
-constexpr int kAssignWarps = 1 + kScorerWarps + kSummerWarps;
+// |x|^2 of the tokens: computed by the scorers from the X tile (and, with
+// kXnormStore, kept per token for the later half-steps of the same side), or
+// loaded from that store (the inputs do not change between half-steps)
+constexpr int kXnormCompute = 0, kXnormStore = 1, kXnormLoad = 2;
+
+constexpr int kScorerWarps = 16;
+constexpr int kAssignWarps = 1 + kScorerWarps;
 constexpr int kAssignThreads = kAssignWarps * 32;
 constexpr int kScorers = kScorerWarps * 32;
-constexpr int kSummers = kSummerWarps * 32;
 constexpr int kTileRows = 128;
-constexpr int kHalfCand = 4;             // candidates kept per column half
-constexpr int kAssignHeader = 16384;     // AssignSmem, keeps the X buffers 1024-aligned
-constexpr int kExtraK = 16;              // the kappa chunk of the MMA
-// named barriers: 1..4 the two scorer warps of a TMEM lane quarter, 5 all scorers
+constexpr int kQuarterCand = 4;      // candidates kept per column quarter
+constexpr int kDeferSlots = 8;       // listed deferred rows per 32 rows of a tile
+constexpr int kDeferCand = 8;        // candidates of a listed deferred row
+constexpr int kDeferAll = 1 << 8;    // defer_count flag: some rows of the group have label -2
+constexpr int kChunkTiles = 16;      // tiles per claimed chunk
+constexpr int kAssignHeader = 12288; // AssignSmem, keeps the X buffers 1024-aligned
+constexpr int kExtraK = 16;          // the kappa chunk of the MMA
+// named barriers: 1..4 the four scorer warps of a TMEM lane quarter, 5 all scorers
 constexpr int kBarScorers = 5;
 
+// A row with several candidates, decided by fixup_kernel.
+struct DeferRec {
+  int32_t tok;
+  int32_t n;                   // candidates listed, ascending
+  int16_t cand[kDeferCand];
+};
+
 struct AssignSmem {
-  uint64_t x_full[2], x_free[2], t_full[2], t_free[2], l_full[2], l_free[2];
+  uint64_t x_full[2], x_free[2], t_full[2], t_free[2];
   uint32_t tmem_base;
   int abort;
+  int claim_h, claim_c;
   float max_nrm;
   float max_kap;
-  float xq[2][kTileRows];                  // |x|^2 per column half's dimensions
-  float mh[2][kTileRows];                  // per-half maxima of u
-  uint8_t kc[2][kTileRows];                // candidates per half (saturating)
-  int16_t cand[2][kTileRows][kHalfCand];
-  // published per tile parity for the summers
-  int16_t lab[2][kTileRows];               // label; -1 not a video token; -2 deferred
-  uint32_t defmask[2][kTileRows / 32];     // deferred rows of the tile, one bit per row
-  int8_t def_n[2][kTileRows];              // deferred row: candidates listed (0 = all)
-  int16_t def_cand[2][kTileRows][2 * kHalfCand];
+  float xq[4][kTileRows];                  // |x|^2 per column quarter's dimensions
+  float mq[4][kTileRows];                  // per-quarter maxima of u
+  uint8_t kc[4][kTileRows];                // candidates per quarter (saturating)
+  int16_t cand[4][kTileRows][kQuarterCand];
 };
 static_assert(sizeof(AssignSmem) <= kAssignHeader, "assign header overflow");
 
@@ -386,128 +399,19 @@ __device__ __forceinline__ uint16_t bf16_bits_rn(float f) {
   return *reinterpret_cast<const uint16_t*>(&b);
 }
 
-// Member sums are fp32: a run of equal labels among a warp's rows of a tile
-// (at most 19 rows, token order) is summed in registers and added with one
-// vector atomic per lane (lane l owns dimensions 4l .. 4l+3, or 2l, 2l+1 for
-// d = 64), so a run costs the L2 one operation per 32-byte sector.
-template <int D>
-__device__ __forceinline__ void flush_row(float* dst, float v0, float v1, float v2, float v3, int lane) {
-  if (D == 128)
-    atomicAdd(reinterpret_cast<float4*>(dst) + lane, make_float4(v0, v1, v2, v3));
-  else
-    atomicAdd(reinterpret_cast<float2*>(dst) + lane, make_float2(v0, v1));
-}
-
-constexpr int kSumRows = (kTileRows + kSummerWarps - 1) / kSummerWarps;  // rows per summer warp
-
-// Decides a deferred row (its candidates listed in ascending j, or all
-// clusters). First, in fp32, t_j = x.(nu_hi + nu_lo)_j + (-kappa_j / 2 in three
-// parts): the products are exact and 16 roundings of at most 2^-24 of the sum
-// of magnitudes are added, so |t_j - u_j| <= 2^-18 |x||nu_j| + 2^-26 |kappa_j|
-// + 2^-20 (|x||nu_j| + |kappa_j| / 2). If one candidate stays within twice that
-// of the maximum it is the answer; otherwise the survivors are re-scored
-// exactly, kappa_j - 2 x.nu_j from the fp64 nu and kappa, ties to the smaller j.
-// One warp; lane owns dimensions 4 lane .. 4 lane + 3 (2 lane, 2 lane + 1 for d = 64):
-// xa holds the first two of them, xb the other two.
-template <int D, int CP>
-__device__ __forceinline__ float approx_t(int j, float x0, float x1, float x2, float x3, const uint8_t* nuh,
-                                         const uint8_t* nul, const uint8_t* kparts, int lane) {
-  auto bf = [](const uint8_t* base, uint32_t off) {
-    return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(base + off)) << 16);
-  };
-  constexpr int kPer = D / 32;  // dimensions per lane (4 or 2), consecutive
-  const uint32_t o0 = sw128_offset(j, kPer * lane, CP);
-  float p = x0 * bf(nuh, o0);
-  p = fmaf(x0, bf(nul, o0), p);
-  p = fmaf(x1, bf(nuh, o0 + 2), p);
-  p = fmaf(x1, bf(nul, o0 + 2), p);
-  if (D == 128) {
-    p = fmaf(x2, bf(nuh, o0 + 4), p);
-    p = fmaf(x2, bf(nul, o0 + 4), p);
-    p = fmaf(x3, bf(nuh, o0 + 6), p);
-    p = fmaf(x3, bf(nul, o0 + 6), p);
-  }
-  for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-  return p + bf(kparts, plain_offset(j, 0)) + bf(kparts, plain_offset(j, 1)) + bf(kparts, plain_offset(j, 2));
-}
-
-template <int D, int CP>
-__device__ __noinline__ int decide_deferred(const AssignSmem* S, int b, int rr, uint32_t xa, uint32_t xb,
-                               const uint8_t* nuh, const uint8_t* nul, const uint8_t* kparts,
-                               float max_nrm, float max_kap, const double* __restrict__ nu_h,
-                               const double* __restrict__ kap_h, int C, int lane) {
-  const float x0 = __uint_as_float(xa << 16), x1 = __uint_as_float(xa & 0xffff0000u);
-  const float x2 = __uint_as_float(xb << 16), x3 = __uint_as_float(xb & 0xffff0000u);
-  float xx = x0 * x0 + x1 * x1 + x2 * x2 + x3 * x3;
-  for (int o = 16; o > 0; o >>= 1) xx += __shfl_xor_sync(0xffffffffu, xx, o);
-  const float E2 = ldexpf(sqrtf(xx) * max_nrm + 0.5f * max_kap, -16);  // twice the bound, with margin
-  const int n = S->def_n[b][rr];
-  constexpr int kMax = 2 * kHalfCand;
-  float t[kMax];
-  float T = -INFINITY;
-  if (n > 0) {  // listed candidates: all evaluated together
-#pragma unroll
-    for (int q = 0; q < kMax; ++q) {
-      t[q] = -INFINITY;
-      if (q < n) t[q] = approx_t<D, CP>(S->def_cand[b][rr][q], x0, x1, x2, x3, nuh, nul, kparts, lane);
-      T = fmaxf(T, t[q]);
-    }
-  } else {
-    for (int j = 0; j < C; ++j) T = fmaxf(T, approx_t<D, CP>(j, x0, x1, x2, x3, nuh, nul, kparts, lane));
-  }
-  int survivors = 0, only = 0;
-  if (n > 0) {
-#pragma unroll
-    for (int q = 0; q < kMax; ++q)
-      if (q < n && t[q] >= T - E2) {
-        ++survivors;
-        only = S->def_cand[b][rr][q];
-      }
-  } else {
-    for (int j = 0; j < C; ++j)
-      if (approx_t<D, CP>(j, x0, x1, x2, x3, nuh, nul, kparts, lane) >= T - E2) {
-        ++survivors;
-        only = j;
-      }
-  }
-  if (survivors == 1) return only;
-  // exact: the survivors in ascending j, strict minimum of kappa_j - 2 x.nu_j
-  const double d0 = x0, d1 = x1, d2 = x2, d3 = x3;
-  double best = INFINITY;
-  int bj = 0;
-  const int J = n > 0 ? n : C;
-  for (int q = 0; q < J; ++q) {
-    const int j = n > 0 ? static_cast<int>(S->def_cand[b][rr][q]) : q;
-    if (approx_t<D, CP>(j, x0, x1, x2, x3, nuh, nul, kparts, lane) < T - E2) continue;
-    const double* nj = nu_h + static_cast<size_t>(j) * D + (D / 32) * lane;
-    const double2 na = *reinterpret_cast<const double2*>(nj);
-    double e = fma(d0, na.x, d1 * na.y);
-    if (D == 128) {
-      const double2 nb = *reinterpret_cast<const double2*>(nj + 2);
-      e = fma(d2, nb.x, fma(d3, nb.y, e));
-    }
-    for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-    const double sc = kap_h[j] - 2.0 * e;
-    if (sc < best) {
-      best = sc;
-      bj = j;
-    }
-  }
-  return bj;
-}
-
-// grid: min(#SMs, B*H*tiles) CTAs, block kAssignThreads. Dynamic smem:
-// [AssignSmem 16 KB][X 2 x 128 x D bf16][nu_hi CP x D][nu_lo CP x D][ones 128 x 16][kappa parts CP x 16]
+// grid: min(#SMs, chunks) CTAs, block kAssignThreads. Dynamic smem:
+// [AssignSmem][X 2 x 128 x D bf16][nu_hi CP x D][nu_lo CP x D][ones 128 x 16][kappa parts CP x 16]
 template <int D, int CP>
 __global__ void __launch_bounds__(kAssignThreads, 1)
-    assign_kernel(const __grid_constant__ CUtensorMap xmap, const uint16_t* __restrict__ x, int N,
-                  int nv, int C, int BH, const uint16_t* __restrict__ nu_hi,
-                  const uint16_t* __restrict__ nu_lo, const double* __restrict__ nu64,
+    assign_kernel(const __grid_constant__ CUtensorMap xmap, int N, int nv, int C, int BH,
+                  const uint16_t* __restrict__ nu_hi, const uint16_t* __restrict__ nu_lo,
                   const double* __restrict__ kappa64, const float* __restrict__ nunorm,
-                  int32_t* __restrict__ assign, float* __restrict__ sums,
-                  int32_t* __restrict__ counts, int* __restrict__ err) {
-  constexpr int kHalfCols = CP / 2;                 // score columns per scorer thread
-  constexpr int kChunks = kHalfCols / 32;           // 32-column TMEM loads per pass
+                  int32_t* __restrict__ head_next, int32_t* __restrict__ assign,
+                  int32_t* __restrict__ defer_count, DeferRec* __restrict__ defer,
+                  float* __restrict__ xnorm, int xnorm_mode, float* __restrict__ head_max,
+                  int* __restrict__ err) {
+  constexpr int kQCols = CP / 4;      // score columns per scorer thread
+  constexpr int kLoads = kQCols / 32;  // 32-column TMEM loads per thread
   constexpr uint32_t kXBytes = kTileRows * D * 2;
   constexpr uint32_t kNuBytes = CP * D * 2;
   static_assert(CP == 128 || CP == 256, "CP must be 128 or 256");
@@ -522,10 +426,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ntiles = (nv + kTileRows - 1) / kTileRows;
-  const long long total = static_cast<long long>(BH) * ntiles;
-  const long long g0 = total * blockIdx.x / gridDim.x;
-  const long long g1 = total * (blockIdx.x + 1) / gridDim.x;
-  if (g0 >= g1) return;
+  const int nchunk = (ntiles + kChunkTiles - 1) / kChunkTiles;
   // the error word can change under us: decide once for the whole CTA
   if (__syncthreads_or(timed_out_before(err) ? 1 : 0)) return;
 
@@ -537,8 +438,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       mbar_init(smem_u32(&S->x_free[b]), kScorerWarps);
       mbar_init(smem_u32(&S->t_full[b]), 1);
       mbar_init(smem_u32(&S->t_free[b]), kScorerWarps);
-      mbar_init(smem_u32(&S->l_full[b]), kScorerWarps / 2);
-      mbar_init(smem_u32(&S->l_free[b]), kSummerWarps);
     }
     fence_mbar_init();
     tma_prefetch_desc(&xmap);
@@ -564,17 +463,31 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   uint32_t tma_par[2] = {0, 0};  // x_full parity each of them completes
   int mma_last = -1;
 
-  long long g = g0;
   int i = 0;  // tiles started by this CTA: selects buffers and barrier phases
-  while (g < g1) {
-    const int h = static_cast<int>(g / ntiles);
-    const int t0 = static_cast<int>(g - static_cast<long long>(h) * ntiles);
-    const int t1 = static_cast<int>(min(static_cast<long long>(ntiles), g1 - static_cast<long long>(h) * ntiles));
+  int cur_h = -1;
+  int h_from = static_cast<int>(static_cast<long long>(blockIdx.x) * BH / gridDim.x);
+  while (true) {
+    if (tid == 0) {  // claim the next chunk: this head first, then the following ones
+      int found = -1, c = 0;
+      for (int k = 0; k < BH && found < 0; ++k) {
+        const int hh = h_from + k < BH ? h_from + k : h_from + k - BH;
+        const int got = atomicAdd(&head_next[hh], 1);
+        if (got < nchunk) {
+          found = hh;
+          c = got;
+        }
+      }
+      S->claim_h = found;
+      S->claim_c = c;
+    }
+    __syncthreads();  // every role is done with the previous chunk
+    if (__syncthreads_or(S->claim_h < 0 || *abort)) break;
+    const int h = S->claim_h;
+    const int t0 = S->claim_c * kChunkTiles, t1 = min(ntiles, t0 + kChunkTiles);
+    h_from = h;
     const int row0 = h * N;
-    __syncthreads();  // every role is done with the previous head
-    if (*abort) break;
-    {  // head h: nu_hi, nu_lo into the swizzled K-major layout of the B operand,
-       // -kappa/2 in three bf16 parts into the kappa chunk, and the bound's maxima
+    if (h != cur_h) {  // head h: nu_hi, nu_lo into the swizzled K-major layout of the B operand,
+                       // -kappa/2 in three bf16 parts into the kappa chunk, and the bound's maxima
       constexpr int chunks = D / 8;
       const uint4* srch = reinterpret_cast<const uint4*>(nu_hi + static_cast<size_t>(h) * CP * D);
       const uint4* srcl = reinterpret_cast<const uint4*>(nu_lo + static_cast<size_t>(h) * CP * D);
@@ -613,11 +526,14 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (lane == 0) {
           S->max_nrm = mn;
           S->max_kap = mk;
+          head_max[2 * h] = mn;  // for fixup_kernel (every CTA of the head writes the same)
+          head_max[2 * h + 1] = mk;
         }
       }
       fence_proxy_async_smem();
+      __syncthreads();
+      cur_h = h;
     }
-    __syncthreads();
 
     if (warp == 0) {
       // ------------------------------------------------------------ producer
@@ -664,12 +580,12 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         }
       }
       __syncwarp();
-    } else if (warp >= kFirstScorer) {
+    } else {
       // ------------------------------------------------------------ scorers
-      const int lq = warp & 3;                   // TMEM lane quarter
-      const int hf = (warp - kFirstScorer) >> 2;  // column half
-      const int r = lq * 32 + lane;              // tile row
-      const int pair_bar = 1 + lq;
+      const int lq = warp & 3;          // TMEM lane quarter
+      const int cq = (warp - 1) >> 2;   // column quarter
+      const int r = lq * 32 + lane;     // tile row
+      const int quad_bar = 1 + lq;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
       const float max_nrm = S->max_nrm, max_kap = S->max_kap;
       for (int tt = t0; tt < t1; ++tt) {
@@ -680,11 +596,18 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
                           mbar_wait(smem_u32(&S->x_full[b]), ph, abort)) ? 0 : 1;
         if (named_sync_or(kBarScorers, kScorers, late)) break;  // every scorer leaves together
         tc_fence_after();
-        {  // |x|^2 over this half of the dimensions; then the X buffer is free
+        const int tok = tt * kTileRows + r;
+        float xsq = 0.f;
+        if (xnorm_mode == kXnormLoad) {
+          // the scorers never read this X tile: it goes back to the producer at once
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&S->x_free[b]));
+          if (tok < nv) xsq = __ldg(xnorm + static_cast<size_t>(h) * nv + tok);
+        } else {  // |x|^2 over this quarter of the dimensions; then the X buffer is free
           const uint8_t* xb = xs + b * kXBytes;
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-          for (int c = hf * (D / 2); c < (hf + 1) * (D / 2); c += 8) {
+          for (int c = cq * (D / 4); c < (cq + 1) * (D / 4); c += 8) {
             const uint4 v = *reinterpret_cast<const uint4*>(xb + sw128_offset(r, c, kTileRows));
             const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xffff0000u);
             const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xffff0000u);
@@ -695,212 +618,112 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
             a2 = fmaf(f2, f2, fmaf(f6, f6, a2));
             a3 = fmaf(f3, f3, fmaf(f7, f7, a3));
           }
-          S->xq[hf][r] = (a0 + a1) + (a2 + a3);
+          S->xq[cq][r] = (a0 + a1) + (a2 + a3);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&S->x_free[b]));
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&S->x_free[b]));
-        // pass 1: maximum of this half's u
-        const uint32_t ta = lane_base + b * CP + hf * kHalfCols;
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < kChunks; c += 2) {  // two chunks per TMEM round trip
-          float v0[32], v1[32];
-          tmem_ld32f(ta + 32 * c, v0);
-          tmem_ld32f(ta + 32 * (c + 1), v1);
-          tmem_wait_ld_f(v0);
-          tmem_wait_ld_f(v1);
-          float m4[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            m4[k] = fmax3(v0[8 * k], v0[8 * k + 1], v0[8 * k + 2]);
-            m4[k] = fmax3(m4[k], v0[8 * k + 3], v0[8 * k + 4]);
-            m4[k] = fmax3(m4[k], v0[8 * k + 5], v0[8 * k + 6]);
-            m4[k] = fmax3(m4[k], v0[8 * k + 7], v1[8 * k]);
-            m4[k] = fmax3(m4[k], v1[8 * k + 1], v1[8 * k + 2]);
-            m4[k] = fmax3(m4[k], v1[8 * k + 3], v1[8 * k + 4]);
-            m4[k] = fmax3(m4[k], v1[8 * k + 5], v1[8 * k + 6]);
-            m4[k] = fmaxf(m4[k], v1[8 * k + 7]);
-          }
-          mx = fmax3(mx, fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        }
-        S->mh[hf][r] = mx;
-        named_sync(pair_bar, 64);
-        // pass 2: candidates within 2E of the row maximum
-        {
-          const float U = fmaxf(S->mh[0][r], S->mh[1][r]);
-          const float xn = sqrtf(S->xq[0][r] + S->xq[1][r]);
-          const float thr = U - ldexpf(xn * max_nrm + 0.5f * max_kap, -12);
-          int k = 0;
-          int16_t cl[kHalfCand] = {0, 0, 0, 0};
-#pragma unroll 1
-          for (int c = 0; c < kChunks; c += 2) {
-            float v0[32], v1[32];
-            tmem_ld32f(ta + 32 * c, v0);
-            tmem_ld32f(ta + 32 * (c + 1), v1);
-            tmem_wait_ld_f(v0);
-            tmem_wait_ld_f(v1);
-            // eight independent partial masks per word keep the OR chains short
-            uint32_t p0[8], p1[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              p0[u] = 0u;
-              p1[u] = 0u;
-            }
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-              p0[q & 7] |= (v0[q] >= thr ? 1u : 0u) << q;
-              p1[q & 7] |= (v1[q] >= thr ? 1u : 0u) << q;
-            }
-            uint32_t bw[2] = {((p0[0] | p0[1]) | (p0[2] | p0[3])) | ((p0[4] | p0[5]) | (p0[6] | p0[7])),
-                              ((p1[0] | p1[1]) | (p1[2] | p1[3])) | ((p1[4] | p1[5]) | (p1[6] | p1[7]))};
-#pragma unroll
-            for (int w2 = 0; w2 < 2; ++w2) {
-              while (bw[w2]) {
-                const int q = __ffs(bw[w2]) - 1;
-                bw[w2] &= bw[w2] - 1;
-                if (k < kHalfCand) cl[k] = static_cast<int16_t>(hf * kHalfCols + 32 * (c + w2) + q);
-                ++k;
-              }
-            }
-          }
-          S->kc[hf][r] = static_cast<uint8_t>(min(k, 255));
-#pragma unroll
-          for (int q = 0; q < kHalfCand; ++q) S->cand[hf][r][q] = cl[q];
-        }
+        // this quarter's scores into registers; then the accumulator is free
+        const uint32_t ta = lane_base + b * CP + cq * kQCols;
+        float v[kQCols];
+        tmem_ld32f(ta, v);
+        if constexpr (kLoads == 2) tmem_ld32f(ta + 32, v + 32);
+        tmem_wait_ld_f(v);
+        if constexpr (kLoads == 2) tmem_wait_ld_f(v + 32);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&S->t_free[b]));
-        named_sync(pair_bar, 64);
-        // the row's decision, published for the summers
-        if (hf == 0) {
-          if (ii >= 2) mbar_wait(smem_u32(&S->l_free[b]), ((ii >> 1) - 1) & 1, abort);
-          const int tok = tt * kTileRows + r;
-          int L = -1;
-          if (tok < nv) {
-            const int k0 = S->kc[0][r], k1 = S->kc[1][r];
-            if (k0 + k1 == 1) L = k0 ? S->cand[0][r][0] : S->cand[1][r][0];
-            if (k0 + k1 != 1 || L >= C) {  // (a padding column only with non-finite input)
-              L = -2;
-              // candidates in ascending j, unless there are too many or one
-              // is a padding column (only with non-finite input)
-              bool listed = k0 + k1 >= 2 && k0 <= kHalfCand && k1 <= kHalfCand;
-              int n = 0;
-              if (listed) {
-                for (int u = 0; u < k0; ++u) S->def_cand[b][r][n++] = S->cand[0][r][u];
-                for (int u = 0; u < k1; ++u) S->def_cand[b][r][n++] = S->cand[1][r][u];
-                for (int u = 0; u < n; ++u) listed = listed && S->def_cand[b][r][u] < C;
-              }
-              S->def_n[b][r] = static_cast<int8_t>(listed ? n : 0);
-            } else {
-              assign[static_cast<size_t>(h) * nv + tok] = L;
-            }
-          }
-          S->lab[b][r] = static_cast<int16_t>(L);
-          // one word per 32 rows: the hf == 0 warps own rows 32 lq .. 32 lq + 31
-          const uint32_t dm = __ballot_sync(0xffffffffu, L == -2);
-          if (lane == 0) S->defmask[b][lq] = dm;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&S->l_full[b]));
-        }
-      }
-    } else {
-      // ------------------------------------------------------------ summers
-      // warp sw owns the contiguous rows [r0, r1) of every tile; all of them
-      // are fetched with one batch of loads, one tile ahead
-      const int sw = warp - kFirstSummer;
-      const int r0 = kTileRows * sw / kSummerWarps, r1 = kTileRows * (sw + 1) / kSummerWarps;
-      const int nr = r1 - r0;
-      const float max_nrm = S->max_nrm, max_kap = S->max_kap;
-      uint32_t wa0[kSumRows], wb0[kSumRows];
-      auto fetch = [&](int tt, uint32_t(&wa)[kSumRows], uint32_t(&wb)[kSumRows]) {
-        const uint16_t* xt = x + (static_cast<size_t>(row0) + static_cast<size_t>(tt) * kTileRows) * D;
+        float m4[4] = {v[0], v[1], v[2], v[3]};
 #pragma unroll
-        for (int k = 0; k < kSumRows; ++k) {
-          wa[k] = 0u;
-          wb[k] = 0u;
-          if (k < nr && tt * kTileRows + r0 + k < nv) {
-            const uint16_t* src = xt + static_cast<size_t>(r0 + k) * D;
-            if (D == 128) {
-              const uint2 v = __ldg(reinterpret_cast<const uint2*>(src) + lane);
-              wa[k] = v.x;
-              wb[k] = v.y;
-            } else {
-              wa[k] = __ldg(reinterpret_cast<const uint32_t*>(src) + lane);
-            }
+        for (int c = 4; c + 7 < kQCols + 4; c += 8) {
+          m4[0] = fmax3(m4[0], v[c], v[c + 1]);
+          m4[1] = fmax3(m4[1], v[c + 2], v[c + 3]);
+          if (c + 4 < kQCols) {
+            m4[2] = fmax3(m4[2], v[c + 4], v[c + 5]);
+            m4[3] = fmax3(m4[3], v[c + 6], v[c + 7]);
           }
         }
-      };
-      auto process = [&](int tt, const uint32_t(&wa)[kSumRows], const uint32_t(&wb)[kSumRows]) -> bool {
-        const int ii = i + (tt - t0), b = ii & 1;
-        if (!mbar_wait(smem_u32(&S->l_full[b]), (ii >> 1) & 1, abort)) return false;
-        // labelled rows: a run of equal labels (token order) is summed in fp32
-        // and added once to the member sums
+        S->mq[cq][r] = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+        named_sync(quad_bar, 128);
+        // candidates of this quarter within 2E of the row maximum
         {
-          int cur = -1, run = 0;
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-          auto flush = [&]() {
-            flush_row<D>(sums + (static_cast<size_t>(h) * C + cur) * D, a0, a1, a2, a3, lane);
-            if (lane == 0) atomicAdd(&counts[h * C + cur], run);
-          };
+          const float U = fmaxf(fmaxf(S->mq[0][r], S->mq[1][r]), fmaxf(S->mq[2][r], S->mq[3][r]));
+          if (xnorm_mode != kXnormLoad) {
+            xsq = (S->xq[0][r] + S->xq[1][r]) + (S->xq[2][r] + S->xq[3][r]);
+            if (xnorm_mode == kXnormStore && cq == 0 && tok < nv) xnorm[static_cast<size_t>(h) * nv + tok] = xsq;
+          }
+          const float thr = U - ldexpf(sqrtf(xsq) * max_nrm + 0.5f * max_kap, -12);
+          int k = 0;
+          int16_t cl[kQuarterCand] = {0, 0, 0, 0};
 #pragma unroll
-          for (int k = 0; k < kSumRows; ++k) {
-            const int L = k < nr ? S->lab[b][r0 + k] : -1;
-            if (L < 0) continue;
-            if (L != cur) {
-              if (cur >= 0) flush();
-              cur = L;
-              run = 0;
-              a0 = a1 = a2 = a3 = 0.f;
-            }
-            ++run;
-            a0 += __uint_as_float(wa[k] << 16);
-            a1 += __uint_as_float(wa[k] & 0xffff0000u);
-            if (D == 128) {
-              a2 += __uint_as_float(wb[k] << 16);
-              a3 += __uint_as_float(wb[k] & 0xffff0000u);
+          for (int w32 = 0; w32 < kLoads; ++w32) {
+            // eight independent partial masks keep the OR chains short
+            uint32_t p8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) p8[u] = 0u;
+#pragma unroll
+            for (int q = 0; q < 32; ++q) p8[q & 7] |= (v[w32 * 32 + q] >= thr ? 1u : 0u) << q;
+            uint32_t bw = ((p8[0] | p8[1]) | (p8[2] | p8[3])) | ((p8[4] | p8[5]) | (p8[6] | p8[7]));
+            while (bw) {
+              const int q = __ffs(bw) - 1;
+              bw &= bw - 1;
+              if (k < kQuarterCand) cl[k] = static_cast<int16_t>(cq * kQCols + 32 * w32 + q);
+              ++k;
             }
           }
-          if (cur >= 0) flush();
-        }
-        // deferred rows (usually none: the scorers' bitmask says which)
-        const uint64_t dm64 = (static_cast<uint64_t>(S->defmask[b][(r0 >> 5) + 1 < kTileRows / 32 ? (r0 >> 5) + 1 : (r0 >> 5)]) << 32) |
-                              S->defmask[b][r0 >> 5];
-        uint32_t mine = static_cast<uint32_t>(dm64 >> (r0 & 31)) & ((nr >= 32 ? 0u : (1u << nr)) - 1u);
-#pragma unroll 1
-        while (mine) {
-          const int k = __ffs(mine) - 1;
-          mine &= mine - 1;
-          const int rr = r0 + k;
-          uint32_t xa = 0u, xb = 0u;  // this row's words (a dynamic pick from the batch)
+          S->kc[cq][r] = static_cast<uint8_t>(min(k, 255));
 #pragma unroll
-          for (int q = 0; q < kSumRows; ++q)
-            if (q == k) {
-              xa = wa[q];
-              xb = wb[q];
-            }
-          const int bj = decide_deferred<D, CP>(S, b, rr, xa, xb, nuh, nul, kparts, max_nrm, max_kap,
-                                                nu64 + static_cast<size_t>(h) * C * D,
-                                                kappa64 + static_cast<size_t>(h) * CP, C, lane);
-          if (lane == 0) {
-            assign[static_cast<size_t>(h) * nv + tt * kTileRows + rr] = bj;
-            atomicAdd(&counts[h * C + bj], 1);
-          }
-          flush_row<D>(sums + (static_cast<size_t>(h) * C + bj) * D, __uint_as_float(xa << 16),
-                       __uint_as_float(xa & 0xffff0000u), __uint_as_float(xb << 16),
-                       __uint_as_float(xb & 0xffff0000u), lane);
+          for (int q = 0; q < kQuarterCand; ++q) S->cand[cq][r][q] = cl[q];
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&S->l_free[b]));
-        return true;
-      };
-      if (t0 < t1) fetch(t0, wa0, wb0);
-      for (int tt = t0; tt < t1; ++tt) {
-        if (!process(tt, wa0, wb0)) break;
-        if (tt + 1 < t1) fetch(tt + 1, wa0, wb0);
+        named_sync(quad_bar, 128);
+        if (cq == 0) {  // the row's decision
+          int L = -3;   // not a video token
+          int total = 0;
+          bool listable = true;
+          if (tok < nv) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int kq = S->kc[q][r];
+              total += kq;
+              listable = listable && kq <= kQuarterCand;
+              // a padding column (only with non-finite input) is never listed
+              for (int u = 0; u < min(kq, kQuarterCand); ++u) listable = listable && S->cand[q][r][u] < C;
+            }
+            if (total == 1) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (S->kc[q][r] == 1) L = S->cand[q][r][0];
+              if (L >= C) L = -2;  // a padding column (only with non-finite input)
+            } else {
+              L = -1;
+            }
+          }
+          const size_t grp = (static_cast<size_t>(h) * ntiles + tt) * 4 + lq;
+          // listed rows get the slots in lane order; the rest are marked -2
+          const unsigned dm = __ballot_sync(0xffffffffu, L == -1 && listable && total <= kDeferCand);
+          const int slot = __popc(dm & ((1u << lane) - 1u));
+          if (L == -1) {
+            if (((dm >> lane) & 1u) && slot < kDeferSlots) {
+              DeferRec rec;
+              rec.tok = tok;
+              rec.n = total;
+              int n = 0;
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                for (int u = 0; u < S->kc[q][r]; ++u) rec.cand[n++] = S->cand[q][r][u];
+              for (; n < kDeferCand; ++n) rec.cand[n] = 0;
+              defer[grp * kDeferSlots + slot] = rec;
+            } else {
+              L = -2;  // too many to list: fixup_kernel compares every cluster
+            }
+          }
+          if (L != -3) assign[static_cast<size_t>(h) * nv + tok] = L;
+          // listed records (at most kDeferSlots), plus kDeferAll if any row has label -2
+          const unsigned all = __ballot_sync(0xffffffffu, L == -2);
+          if (lane == 0) defer_count[grp] = min(__popc(dm), kDeferSlots) | (all ? kDeferAll : 0);
+        }
       }
     }
     i += t1 - t0;
-    g += t1 - t0;
   }
   __syncthreads();
   if (*abort && tid == 0) {
@@ -916,22 +739,384 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 2 * CP);
 }
 
+// ---------------------------------------------------------------- fixup
+//
+// Decides the rows the scorers could not: the listed deferred rows of every
+// (tile, 32-row group) and the rows labelled -2. One warp per group; lane l
+// holds dimensions (D/32) l .. (D/32) l + D/32 - 1 of the row. First, in fp32,
+// t_j = x.(nu_hi + nu_lo)_j - kappa_j / 2: the products are exact, and the
+// sums and the rounded -kappa_j/2 err by far less than
+// 2^-17 (|x||nu_j| + |kappa_j|), so every j within
+// E2 = 2^-16 (|x| max|nu| + max|kappa| / 2) of the best t survives; one
+// survivor is the answer; otherwise the survivors are re-scored exactly,
+// kappa_j - 2 x.nu_j from the fp64 nu and kappa, ties to the smaller j.
+template <int D, int CP>
+__device__ float approx_score(const uint16_t* __restrict__ hi, const uint16_t* __restrict__ lo,
+                              const double* __restrict__ kap, int j, const float* xv, int lane) {
+  constexpr int kPer = D / 32;
+  const size_t o = static_cast<size_t>(j) * D + kPer * lane;
+  float p = 0.f;
+  if (kPer == 4) {
+    const uint2 h2 = __ldg(reinterpret_cast<const uint2*>(hi + o));
+    const uint2 l2 = __ldg(reinterpret_cast<const uint2*>(lo + o));
+    p = fmaf(xv[0], __uint_as_float(h2.x << 16), p);
+    p = fmaf(xv[0], __uint_as_float(l2.x << 16), p);
+    p = fmaf(xv[1], __uint_as_float(h2.x & 0xffff0000u), p);
+    p = fmaf(xv[1], __uint_as_float(l2.x & 0xffff0000u), p);
+    p = fmaf(xv[2], __uint_as_float(h2.y << 16), p);
+    p = fmaf(xv[2], __uint_as_float(l2.y << 16), p);
+    p = fmaf(xv[3], __uint_as_float(h2.y & 0xffff0000u), p);
+    p = fmaf(xv[3], __uint_as_float(l2.y & 0xffff0000u), p);
+  } else {
+    const uint32_t h1 = __ldg(reinterpret_cast<const uint32_t*>(hi + o));
+    const uint32_t l1 = __ldg(reinterpret_cast<const uint32_t*>(lo + o));
+    p = fmaf(xv[0], __uint_as_float(h1 << 16), p);
+    p = fmaf(xv[0], __uint_as_float(l1 << 16), p);
+    p = fmaf(xv[1], __uint_as_float(h1 & 0xffff0000u), p);
+    p = fmaf(xv[1], __uint_as_float(l1 & 0xffff0000u), p);
+  }
+  for (int s = 16; s > 0; s >>= 1) p += __shfl_xor_sync(0xffffffffu, p, s);
+  return p + static_cast<float>(-0.5 * kap[j]);
+}
+
+template <int D>
+__device__ __forceinline__ void load_row(const uint16_t* __restrict__ xrow, float* xv, int lane) {
+  xv[0] = xv[1] = xv[2] = xv[3] = 0.f;
+  if (D == 128) {
+    const uint2 w = __ldg(reinterpret_cast<const uint2*>(xrow) + lane);
+    xv[0] = __uint_as_float(w.x << 16);
+    xv[1] = __uint_as_float(w.x & 0xffff0000u);
+    xv[2] = __uint_as_float(w.y << 16);
+    xv[3] = __uint_as_float(w.y & 0xffff0000u);
+  } else {
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(xrow) + lane);
+    xv[0] = __uint_as_float(w << 16);
+    xv[1] = __uint_as_float(w & 0xffff0000u);
+  }
+}
+
+// exact score kappa_j - 2 x.nu_j in fp64 (whole warp)
+template <int D>
+__device__ __forceinline__ double exact_score(const double* __restrict__ nu64h, const double* __restrict__ kap,
+                                              int j, const float* xv, int lane) {
+  constexpr int kPer = D / 32;
+  const double* nj = nu64h + static_cast<size_t>(j) * D + kPer * lane;
+  double e = 0.0;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) e = fma(static_cast<double>(xv[u]), nj[u], e);
+  for (int s = 16; s > 0; s >>= 1) e += __shfl_xor_sync(0xffffffffu, e, s);
+  return kap[j] - 2.0 * e;
+}
+
+// The label of one row from its listed candidates (n >= 1, ascending): the
+// fp32 scores decide when one candidate stays within E2 of the best,
+// otherwise the survivors are compared exactly (ties to the smaller j).
+template <int D, int CP>
+__device__ int decide_listed(const float* xv, const uint16_t* __restrict__ hi, const uint16_t* __restrict__ lo,
+                             const double* __restrict__ nu64h, const double* __restrict__ kap, float E2,
+                             const int16_t* cand, int n, int lane) {
+  float t[kDeferCand];
+  float T = -INFINITY;
+#pragma unroll
+  for (int q = 0; q < kDeferCand; ++q) {
+    t[q] = q < n ? approx_score<D, CP>(hi, lo, kap, cand[q], xv, lane) : -INFINITY;
+    T = fmaxf(T, t[q]);
+  }
+  int survivors = 0, only = 0;
+#pragma unroll
+  for (int q = 0; q < kDeferCand; ++q)
+    if (q < n && t[q] >= T - E2) {
+      ++survivors;
+      only = cand[q];
+    }
+  if (survivors == 1) return only;
+  double best = INFINITY;
+  int bj = 0;
+#pragma unroll
+  for (int q = 0; q < kDeferCand; ++q) {
+    if (q >= n || t[q] < T - E2) continue;
+    const double sc = exact_score<D>(nu64h, kap, cand[q], xv, lane);
+    if (sc < best) {
+      best = sc;
+      bj = cand[q];
+    }
+  }
+  return bj;
+}
+
+// The label of a row against every cluster (rows whose candidates were not
+// listed): each lane scores its clusters j = lane, lane + 32, ... exactly,
+// kappa_j - 2 x.nu_j in fp64 over the whole row, then the warp takes the
+// minimum, ties to the smaller j.
+template <int D>
+__device__ int decide_all(const uint16_t* __restrict__ xrow, const double* __restrict__ nu64h,
+                          const double* __restrict__ kap, int C, int lane) {
+  double best = INFINITY;
+  int bj = 0x7fffffff;
+  for (int j = lane; j < C; j += 32) {
+    const double* nj = nu64h + static_cast<size_t>(j) * D;
+    double e[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+    for (int i = 0; i < D; i += 8) {
+      const uint4 xw = __ldg(reinterpret_cast<const uint4*>(xrow + i));
+      const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const double2 nv = __ldg(reinterpret_cast<const double2*>(nj + i + 2 * u));
+        e[u] = fma(static_cast<double>(__uint_as_float(w[u] << 16)), nv.x, e[u]);
+        e[u] = fma(static_cast<double>(__uint_as_float(w[u] & 0xffff0000u)), nv.y, e[u]);
+      }
+    }
+    const double sc = kap[j] - 2.0 * ((e[0] + e[1]) + (e[2] + e[3]));
+    if (sc < best) {  // j ascends within a lane
+      best = sc;
+      bj = j;
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+    if (ob < best || (ob == best && oj < bj)) {
+      best = ob;
+      bj = oj;
+    }
+  }
+  return bj;
+}
+
+// E2 = 2^-16 (|x| max|nu| + max|kappa| / 2) of a row (whole warp)
+__device__ __forceinline__ float row_e2(const float* xv, float max_nrm, float max_kap) {
+  float xx = xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
+  for (int s = 16; s > 0; s >>= 1) xx += __shfl_xor_sync(0xffffffffu, xx, s);
+  return ldexpf(sqrtf(xx) * max_nrm + 0.5f * max_kap, -16);
+}
+
+// grid: ceil(BH * ntiles * 4 / 8) blocks of 8 warps, one warp per (head, tile, 32-row group)
+template <int D, int CP>
+__global__ void __launch_bounds__(256)
+    fixup_kernel(const uint16_t* __restrict__ x, int N, int nv, int C, int BH, int ntiles,
+                 const uint16_t* __restrict__ nu_hi, const uint16_t* __restrict__ nu_lo,
+                 const double* __restrict__ nu64, const double* __restrict__ kappa64,
+                 const float* __restrict__ head_max, int32_t* __restrict__ assign,
+                 const int32_t* __restrict__ defer_count, const DeferRec* __restrict__ defer,
+                 int* __restrict__ err) {
+  const int lane = threadIdx.x & 31;
+  if (timed_out_before(err)) return;  // the scorers may not have written their lists
+  const long long grp = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (grp >= static_cast<long long>(BH) * ntiles * 4) return;
+  const int dc = defer_count[grp];
+  if (dc == 0) return;  // (warp-uniform) nothing was deferred in these 32 rows
+  const int n_def = min(dc & (kDeferAll - 1), kDeferSlots);
+  const int h = static_cast<int>(grp / (static_cast<long long>(ntiles) * 4));
+  const int rem = static_cast<int>(grp - static_cast<long long>(h) * ntiles * 4);
+  const int tt = rem >> 2, lq = rem & 3;
+  const float mn = head_max[2 * h], mk = head_max[2 * h + 1];
+  const uint16_t* hi = nu_hi + static_cast<size_t>(h) * CP * D;
+  const uint16_t* lo = nu_lo + static_cast<size_t>(h) * CP * D;
+  const double* nuh = nu64 + static_cast<size_t>(h) * C * D;
+  const double* kap = kappa64 + static_cast<size_t>(h) * CP;
+  int32_t* asg = assign + static_cast<size_t>(h) * nv;
+  const uint16_t* xh = x + static_cast<size_t>(h) * N * D;
+  // listed rows
+  for (int s = 0; s < n_def; ++s) {
+    const DeferRec& rec = defer[grp * kDeferSlots + s];
+    const int tok = rec.tok;
+    if (tok < 0 || tok >= nv) continue;
+    const int n = min(max(rec.n, 1), kDeferCand);
+    int16_t cand[kDeferCand];
+    bool valid = true;  // a list that does not look right falls back to every cluster
+#pragma unroll
+    for (int q = 0; q < kDeferCand; ++q) {
+      cand[q] = rec.cand[q];
+      valid = valid && (q >= n || (cand[q] >= 0 && cand[q] < C));
+    }
+    int lbl;
+    if (valid) {
+      float xv[4];
+      load_row<D>(xh + static_cast<size_t>(tok) * D, xv, lane);
+      lbl = decide_listed<D, CP>(xv, hi, lo, nuh, kap, row_e2(xv, mn, mk), cand, n, lane);
+    } else {
+      lbl = decide_all<D>(xh + static_cast<size_t>(tok) * D, nuh, kap, C, lane);
+    }
+    if (lane == 0) asg[tok] = lbl;
+  }
+  // rows whose candidates could not be listed: every cluster
+  if (!(dc & kDeferAll)) return;
+  const int tok = tt * kTileRows + lq * 32 + lane;
+  unsigned all = __ballot_sync(0xffffffffu, tok < nv && asg[tok] == -2);
+  while (all) {
+    const int l = __ffs(all) - 1;
+    all &= all - 1;
+    const int t = tt * kTileRows + lq * 32 + l;
+    const int lbl = decide_all<D>(xh + static_cast<size_t>(t) * D, nuh, kap, C, lane);
+    if (lane == 0) asg[t] = lbl;
+  }
+}
+
+// ---------------------------------------------------------------- update
+//
+// Member sums are exact: components with |x| < 2^-24 count as zero, so every
+// partial sum is a multiple of 2^-31 below 2^22 in magnitude and fp64 holds it
+// exactly; the order of the additions (and of the fp64 atomic additions of
+// partial sums) changes nothing, and the centroid fp32(sum / n) is the one the
+// exact mean rounds to.
+
+constexpr int kMaxClusters = 256;
+constexpr int kUpdTokens = 2048;     // consecutive tokens per CTA
+constexpr int kUpdThreads = 256;
+constexpr int kUpdWarps = kUpdThreads / 32;
+
+__device__ __forceinline__ double flushed(float v) {
+  return fabsf(v) < 5.9604644775390625e-08f ? 0.0 : static_cast<double>(v);  // 2^-24
+}
+
+__device__ __forceinline__ void red_f64(double* dst, double v) {
+  asm volatile("red.global.add.f64 [%0], %1;" ::"l"(dst), "d"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_s32(int32_t* dst, int v) {
+  asm volatile("red.global.add.s32 [%0], %1;" ::"l"(dst), "r"(v) : "memory");
+}
+
+// grid (ceil(nv / kUpdTokens), BH), block kUpdThreads. The CTA groups its
+// kUpdTokens consecutive tokens by label in shared memory (the order inside a
+// cluster is irrelevant: the sums are exact), adds its member counts to
+// counts[h][j], and each warp sums a contiguous run of the grouped order in
+// fp64, adding every cluster's partial sum to sums[h][j]. The rows it reads
+// all lie in the chunk's own contiguous slice of X.
+template <int D>
+__global__ void __launch_bounds__(kUpdThreads)
+    update_kernel(const uint16_t* __restrict__ x, int N, int nv, int C,
+                  const int32_t* __restrict__ assign, double* __restrict__ sums,
+                  int32_t* __restrict__ counts, int* __restrict__ err) {
+  constexpr int kPer = D / 32;
+  constexpr int kBatch = 16;
+  __shared__ int cnt[kMaxClusters];
+  __shared__ int base[kMaxClusters + 1];
+  __shared__ int16_t order[kUpdTokens];
+  const int h = blockIdx.y, c0 = blockIdx.x * kUpdTokens;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (timed_out_before(err)) return;  // labels of an aborted step are not to be trusted
+  const int n = min(kUpdTokens, nv - c0);
+  const int32_t* a = assign + static_cast<size_t>(h) * nv + c0;
+  for (int j = tid; j < C; j += kUpdThreads) cnt[j] = 0;
+  __syncthreads();
+  for (int t = tid; t < n; t += kUpdThreads) {
+    const int l = a[t];
+    if (l >= 0 && l < C) atomicAdd(&cnt[l], 1);
+    else report_error(err, kErrBadLabel);
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of the counts
+    int run = 0;
+    for (int j0 = 0; j0 < C; j0 += 32) {
+      const int j = j0 + lane;
+      const int c = j < C ? cnt[j] : 0;
+      int incl = c;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (j < C) base[j] = run + incl - c;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) base[C] = run;
+  }
+  __syncthreads();
+  for (int j = tid; j < C; j += kUpdThreads) {
+    if (cnt[j] > 0) red_s32(&counts[static_cast<size_t>(h) * C + j], cnt[j]);
+  }
+  __syncthreads();
+  for (int j = tid; j < C; j += kUpdThreads) cnt[j] = 0;
+  __syncthreads();
+  for (int t = tid; t < n; t += kUpdThreads) {
+    const int l = a[t];
+    if (l >= 0 && l < C) order[base[l] + atomicAdd(&cnt[l], 1)] = static_cast<int16_t>(t);
+  }
+  __syncthreads();
+  const int nvalid = base[C];
+  const int p0 = warp * nvalid / kUpdWarps, p1 = (warp + 1) * nvalid / kUpdWarps;
+  if (p0 >= p1) return;
+  // the cluster of position p0: the last j with base[j] <= p0
+  int lo_j = 0, hi_j = C - 1;
+  while (lo_j < hi_j) {
+    const int mid = (lo_j + hi_j + 1) >> 1;
+    if (base[mid] <= p0) lo_j = mid;
+    else hi_j = mid - 1;
+  }
+  int j = lo_j, end = base[j + 1];
+  const uint16_t* xc = x + (static_cast<size_t>(h) * N + c0) * D;
+  double acc[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) acc[u] = 0.0;
+  bool any = false;
+  auto flush = [&]() {
+    if (any) {
+      double* dst = sums + (static_cast<size_t>(h) * C + j) * D + kPer * lane;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) red_f64(dst + u, acc[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) acc[u] = 0.0;
+    any = false;
+  };
+  for (int pb = p0; pb < p1; pb += kBatch) {
+    uint32_t w0[kBatch], w1[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {  // the batch's rows in flight together
+      w0[q] = 0u;
+      w1[q] = 0u;
+      if (pb + q < p1) {
+        const int t = order[pb + q];
+        if (kPer == 4) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2*>(xc + static_cast<size_t>(t) * D) + lane);
+          w0[q] = v.x;
+          w1[q] = v.y;
+        } else {
+          w0[q] = __ldg(reinterpret_cast<const uint32_t*>(xc + static_cast<size_t>(t) * D) + lane);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+      const int p = pb + q;
+      if (p >= p1) break;
+      while (p >= end && j + 1 < C) {  // next non-empty cluster
+        flush();
+        ++j;
+        end = base[j + 1];
+      }
+      acc[0] += flushed(__uint_as_float(w0[q] << 16));
+      acc[1] += flushed(__uint_as_float(w0[q] & 0xffff0000u));
+      if (kPer == 4) {
+        acc[2] += flushed(__uint_as_float(w1[q] << 16));
+        acc[3] += flushed(__uint_as_float(w1[q] & 0xffff0000u));
+      }
+      any = true;
+    }
+  }
+  flush();
+}
+
 // ---------------------------------------------------------------- finalize
 
-// grid (C, BH), block d.
-__global__ void finalize_kernel(float* __restrict__ sums, int32_t* __restrict__ counts,
-                                float* __restrict__ cent, int32_t* __restrict__ sizes, int C,
-                                int d) {
+// grid (C, BH), block d: centroid = fp32(sum / n) (IEEE fp64 division, one
+// rounding), an empty cluster keeps its centroid; clears the sums and the
+// chunk counters for the next half-step.
+__global__ void finalize_kernel(double* __restrict__ sums, int32_t* __restrict__ counts,
+                                float* __restrict__ cent, int32_t* __restrict__ sizes,
+                                int32_t* __restrict__ head_next, int C, int d) {
   const int h = blockIdx.y, j = blockIdx.x, i = threadIdx.x;
   const int n = counts[h * C + j];
-  const size_t o = (static_cast<size_t>(h) * C + j) * d + i;
-  if (n > 0) cent[o] = static_cast<float>(static_cast<double>(sums[o]) / static_cast<double>(n));
-  sums[o] = 0.f;
+  const size_t e = (static_cast<size_t>(h) * C + j) * d + i;
+  if (n > 0) cent[e] = static_cast<float>(sums[e] / static_cast<double>(n));
+  sums[e] = 0.0;
   __syncthreads();
   if (i == 0) {
     sizes[h * C + j] = n;
     counts[h * C + j] = 0;
   }
+  if (i == 0 && j == 0) head_next[h] = 0;
 }
 
 // ---------------------------------------------------------------- host side
@@ -946,17 +1131,23 @@ struct StepWs {
   double* kappa64;
   float* kappa;
   float* nunorm;
-  float* sums;
+  double* sums;
   int32_t* counts;
+  int32_t* head_next;
+  float* head_max;
+  float* xnorm;
+  int32_t* defer_count;
+  DeferRec* defer;
 };
 
 // columns of the scoring MMA: the cluster count padded so that four threads
 // per row read one or two 32-column TMEM chunks each
 inline int score_cols(int c) { return c <= 128 ? 128 : 256; }
 
-size_t carve_step(void* ws, int BH, int d, int Cmax, StepWs* out) {
+size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out) {
   Carver cv(ws);
   const int CP = score_cols(Cmax);
+  const size_t ntiles = (static_cast<size_t>(nv) + kTileRows - 1) / kTileRows;
   StepWs w;
   w.M = cv.take<double>(static_cast<size_t>(BH) * d * d);
   w.nu64 = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
@@ -965,15 +1156,21 @@ size_t carve_step(void* ws, int BH, int d, int Cmax, StepWs* out) {
   w.kappa64 = cv.take<double>(static_cast<size_t>(BH) * CP);
   w.kappa = cv.take<float>(static_cast<size_t>(BH) * CP);
   w.nunorm = cv.take<float>(static_cast<size_t>(BH) * CP);
-  w.sums = cv.take<float>(static_cast<size_t>(BH) * Cmax * d);
+  w.sums = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
   w.counts = cv.take<int32_t>(static_cast<size_t>(BH) * Cmax);
+  w.head_next = cv.take<int32_t>(static_cast<size_t>(BH));
+  w.head_max = cv.take<float>(static_cast<size_t>(BH) * 2);
+  w.xnorm = cv.take<float>(static_cast<size_t>(BH) * nv);
+  w.defer_count = cv.take<int32_t>(static_cast<size_t>(BH) * ntiles * 4);
+  w.defer = cv.take<DeferRec>(static_cast<size_t>(BH) * ntiles * 4 * kDeferSlots);
   if (out) *out = w;
   return cv.used + 256;
 }
 
 template <int D, int CP>
 svoo_status launch_assign(const CUtensorMap& xmap, const svoo_shape* sh, const void* x, int C,
-                          const StepWs& w, int32_t* assign, int32_t* dev_err, cudaStream_t st) {
+                          const StepWs& w, int32_t* assign, float* xnorm, int xnorm_mode,
+                          int32_t* dev_err, cudaStream_t st) {
   const int BH = bh_of(sh), N = sh->N, nv = nvideo_of(sh);
   const size_t smem = 1024 + kAssignHeader + 2 * static_cast<size_t>(kTileRows) * D * 2 +
                       2 * static_cast<size_t>(CP) * D * 2 + (kTileRows + CP) * kExtraK * 2;
@@ -984,26 +1181,39 @@ svoo_status launch_assign(const CUtensorMap& xmap, const svoo_shape* sh, const v
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return SVOO_ERR_CUDA;
-  const long long total = static_cast<long long>(BH) * ((nv + kTileRows - 1) / kTileRows);
-  const int grid = static_cast<int>(total < sms ? total : sms);
+  const int ntiles = (nv + kTileRows - 1) / kTileRows;
+  const long long chunks = static_cast<long long>(BH) * ((ntiles + kChunkTiles - 1) / kChunkTiles);
+  const int grid = static_cast<int>(chunks < sms ? chunks : sms);
   assign_kernel<D, CP><<<grid, kAssignThreads, smem, st>>>(
-      xmap, static_cast<const uint16_t*>(x), N, nv, C, BH, w.nu_hi, w.nu_lo, w.nu64, w.kappa64,
-      w.nunorm, assign, w.sums, w.counts, dev_err);
+      xmap, N, nv, C, BH, w.nu_hi, w.nu_lo, w.kappa64, w.nunorm, w.head_next, assign,
+      w.defer_count, w.defer, xnorm, xnorm_mode, w.head_max, dev_err);
+  if (cudaGetLastError() != cudaSuccess) return SVOO_ERR_CUDA;
+  const long long groups = static_cast<long long>(BH) * ntiles * 4;
+  fixup_kernel<D, CP><<<static_cast<unsigned>((groups + 7) / 8), 256, 0, st>>>(
+      static_cast<const uint16_t*>(x), N, nv, C, BH, ntiles, w.nu_hi, w.nu_lo, w.nu64, w.kappa64,
+      w.head_max, assign, w.defer_count, w.defer, dev_err);
+  if (cudaGetLastError() != cudaSuccess) return SVOO_ERR_CUDA;
+  update_kernel<D><<<dim3((nv + kUpdTokens - 1) / kUpdTokens, BH), kUpdThreads, 0, st>>>(
+      static_cast<const uint16_t*>(x), N, nv, C, assign, w.sums, w.counts, dev_err);
   return SVOO_OK;
 }
 
-// One half-step. metric_cent == nullptr: identity metric.
+// One half-step. metric_cent == nullptr: identity metric. xnorm: per-token
+// |x|^2 store of this side (xnorm_mode kXnormStore / kXnormLoad), else the
+// step computes |x|^2 itself.
 svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, int32_t* sizes,
                      int32_t* assign, const float* metric_cent, const int32_t* metric_sizes,
                      int metric_C, const StepWs& w, int32_t* dev_err, cudaStream_t st,
-                     int zero_C) {
+                     int zero_C, float* xnorm = nullptr, int xnorm_mode = kXnormCompute) {
   const int BH = bh_of(sh), d = sh->d, N = sh->N;
   const int CP = score_cols(C);
   // finalize_kernel re-zeroes what a step used, so only the first step of a
-  // call clears the accumulators (for the largest cluster count of the call).
+  // call clears the sums and the chunk counters (for the call's largest
+  // cluster count).
   if (zero_C > 0) {
-    if (cudaMemsetAsync(w.sums, 0, sizeof(float) * BH * static_cast<size_t>(zero_C) * d, st) != cudaSuccess ||
-        cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * BH * static_cast<size_t>(zero_C), st) != cudaSuccess)
+    if (cudaMemsetAsync(w.sums, 0, sizeof(double) * BH * static_cast<size_t>(zero_C) * d, st) != cudaSuccess ||
+        cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * BH * static_cast<size_t>(zero_C), st) != cudaSuccess ||
+        cudaMemsetAsync(w.head_next, 0, sizeof(int32_t) * BH, st) != cudaSuccess)
       return SVOO_ERR_CUDA;
   }
   if (metric_cent) {
@@ -1023,19 +1233,36 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
   CUtensorMap xmap;
   if (encode_tiled_2d(&xmap, x, static_cast<uint64_t>(BH) * N, d, kTileRows, 64) != CUDA_SUCCESS)
     return SVOO_ERR_CUDA;
+  if (!xnorm) {  // a lone half-step computes |x|^2 from the tiles
+    xnorm = w.xnorm;
+    xnorm_mode = kXnormCompute;
+  }
   svoo_status s;
   if (d == 128)
-    s = CP == 256 ? launch_assign<128, 256>(xmap, sh, x, C, w, assign, dev_err, st)
-                  : launch_assign<128, 128>(xmap, sh, x, C, w, assign, dev_err, st);
+    s = CP == 256 ? launch_assign<128, 256>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, dev_err, st)
+                  : launch_assign<128, 128>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, dev_err, st);
   else
-    s = CP == 256 ? launch_assign<64, 256>(xmap, sh, x, C, w, assign, dev_err, st)
-                  : launch_assign<64, 128>(xmap, sh, x, C, w, assign, dev_err, st);
+    s = CP == 256 ? launch_assign<64, 256>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, dev_err, st)
+                  : launch_assign<64, 128>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, dev_err, st);
   if (s != SVOO_OK) return s;
-  finalize_kernel<<<dim3(C, BH), d, 0, st>>>(w.sums, w.counts, cent, sizes, C, d);
+  finalize_kernel<<<dim3(C, BH), d, 0, st>>>(w.sums, w.counts, cent, sizes, w.head_next, C, d);
   return launch_status();
 }
 
 bool cluster_counts_ok(int C) { return C >= 1 && C <= 256; }
+
+// Workspace of a whole svoo_cluster call: one half-step's scratch, then the
+// per-token |x|^2 of the queries and of the keys (fp32 [BH][N - n_text] each).
+size_t carve_call(void* ws, const svoo_shape* sh, int Cmax, StepWs* w, float** xn_q, float** xn_k) {
+  const size_t step = carve_step(ws, bh_of(sh), sh->d, Cmax, nvideo_of(sh), w);
+  Carver cv(ws ? static_cast<char*>(ws) + step : nullptr);
+  const size_t n = static_cast<size_t>(bh_of(sh)) * nvideo_of(sh);
+  float* a = cv.take<float>(n);
+  float* b = cv.take<float>(n);
+  if (xn_q) *xn_q = a;
+  if (xn_k) *xn_k = b;
+  return step + cv.used + 256;
+}
 
 // Cluster count that sizes a half-step's scratch: metric_C only counts when a
 // metric is given (it is ignored, whatever its value, for the identity).
@@ -1050,7 +1277,7 @@ using namespace svoo;
 
 extern "C" size_t svoo_cluster_workspace_size(const svoo_shape* shape, int n_qc, int n_kc) {
   if (!shape_ok(shape) || !cluster_counts_ok(n_qc) || !cluster_counts_ok(n_kc)) return 0;
-  return carve_step(nullptr, bh_of(shape), shape->d, n_qc > n_kc ? n_qc : n_kc, nullptr);
+  return carve_call(nullptr, shape, n_qc > n_kc ? n_qc : n_kc, nullptr, nullptr, nullptr);
 }
 
 extern "C" svoo_status svoo_cluster_step(const svoo_shape* shape, const void* x, int C, float* cent,
@@ -1063,7 +1290,7 @@ extern "C" svoo_status svoo_cluster_step(const svoo_shape* shape, const void* x,
   if (!aligned(x, 16)) return SVOO_ERR_INVALID_ARG;
   const int BH = bh_of(shape);
   StepWs w;
-  size_t need = carve_step(workspace, BH, shape->d, step_clusters(C, metric_cent, metric_C), &w);
+  size_t need = carve_step(workspace, BH, shape->d, step_clusters(C, metric_cent, metric_C), nvideo_of(shape), &w);
   if (workspace_bytes < need) return SVOO_ERR_WORKSPACE;
   return run_step(shape, x, C, cent, sizes, assign, metric_cent, metric_sizes, metric_C, w, dev_err,
                   static_cast<cudaStream_t>(stream), C);
@@ -1085,7 +1312,8 @@ extern "C" svoo_status svoo_cluster(const svoo_shape* shape, const void* q, cons
   if (!aligned(q, 16) || !aligned(k, 16)) return SVOO_ERR_INVALID_ARG;
   const int BH = bh_of(shape), d = shape->d, N = shape->N, nv = nvideo_of(shape);
   StepWs w;
-  size_t need = carve_step(workspace, BH, d, n_qc > n_kc ? n_qc : n_kc, &w);
+  float *xn_q = nullptr, *xn_k = nullptr;
+  size_t need = carve_call(workspace, shape, n_qc > n_kc ? n_qc : n_kc, &w, &xn_q, &xn_k);
   if (workspace_bytes < need) return SVOO_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!warm) {
@@ -1095,11 +1323,12 @@ extern "C" svoo_status svoo_cluster(const svoo_shape* shape, const void* q, cons
   const int Cmax = n_qc > n_kc ? n_qc : n_kc;
   for (int it = 0; it < iters; ++it) {
     const bool ident = identity || (it == 0 && !warm);
+    const int xmode = it == 0 ? kXnormStore : kXnormLoad;  // inputs fixed for the whole call
     svoo_status s = run_step(shape, q, n_qc, q_cent, q_sizes, q_assign, ident ? nullptr : k_cent,
-                             k_sizes, n_kc, w, dev_err, st, it == 0 ? Cmax : 0);
+                             k_sizes, n_kc, w, dev_err, st, it == 0 ? Cmax : 0, xn_q, xmode);
     if (s != SVOO_OK) return s;
     s = run_step(shape, k, n_kc, k_cent, k_sizes, k_assign, identity ? nullptr : q_cent, q_sizes,
-                 n_qc, w, dev_err, st, 0);
+                 n_qc, w, dev_err, st, 0, xn_k, xmode);
     if (s != SVOO_OK) return s;
   }
   return SVOO_OK;
@@ -1161,13 +1390,13 @@ extern "C" svoo_status svoo_cluster_step_static(const svoo_shape* shape, const v
   if (!aligned(x, 16)) return SVOO_ERR_INVALID_ARG;
   const int BH = bh_of(shape);
   const int Cmax = step_clusters(C, metric_cent, metric_C);
-  if (carve_step(nullptr, BH, shape->d, Cmax, nullptr) > kStaticScratchBytes)
+  if (carve_step(nullptr, BH, shape->d, Cmax, nvideo_of(shape), nullptr) > kStaticScratchBytes)
     return SVOO_ERR_WORKSPACE;  // shape needs more than the fixed scratch holds
   int dev = 0;
   void* base = scratch_address(&dev);
   if (!base) return SVOO_ERR_CUDA;
   StepWs w;
-  carve_step(base, BH, shape->d, Cmax, &w);
+  carve_step(base, BH, shape->d, Cmax, nvideo_of(shape), &w);
   return run_step(shape, x, C, cent, sizes, assign, metric_cent, metric_sizes, metric_C, w, dev_err,
                   static_cast<cudaStream_t>(stream), C);
 }

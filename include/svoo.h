@@ -51,10 +51,10 @@
  *  - Limits: 1 <= B*H <= 65535, B*H*N < 2^31 - 256, 1 <= N - n_text, N <= 2^20,
  *    d in {64, 128},
  *    1 <= n_qc, n_kc <= 256, block_q in {64, 128}, 0 <= n_text, iters >= 1.
- *    Inputs must be finite. Centroid member sums are fp32 (runs of at most
- *    19 consecutive same-cluster tokens summed in registers, the run sums
- *    added atomically), so a centroid lies within (n + 18) 2^-24 mean|x| of
- *    the exact mean of its n members.
+ *    Inputs must be finite. Centroid member sums are exact (fp64, with
+ *    components |x| < 2^-24 counted as zero, so every partial sum is a
+ *    multiple of 2^-31 below 2^22), and a centroid is its exact mean rounded
+ *    once to fp32, whatever the order in which the GPU added the members.
  */
 #ifndef SVOO_H
 #define SVOO_H
@@ -145,9 +145,8 @@ size_t svoo_cluster_workspace_size(const svoo_shape *shape, int n_qc, int n_kc);
  * (with kappa folded in); when more than one cluster lies within the MMA's
  * error bound of the best, those candidates are compared again, closer, and
  * in fp64 when still within bound, so the result is that of an fp64
- * evaluation. Update: member means from fp32 sums (see the limits above; the
- * rounding of the sums follows the order of the atomic additions, so two
- * runs can differ in the last bits of a centroid); an empty cluster keeps its
+ * evaluation. Update: member means from exact sums (see the limits above), so
+ * equal labels give bit-identical centroids; an empty cluster keeps its
  * centroid. */
 svoo_status svoo_cluster(const svoo_shape *shape, const void *q, const void *k, int n_qc,
                          int n_kc, int iters, int flags, int32_t *q_assign, int32_t *k_assign,

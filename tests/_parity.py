@@ -59,34 +59,23 @@ def check_assign(gpu_assign, o_assign, best, second, what=""):
     return agree, int(diff.sum())
 
 
-# Centroid update: the GPU sums each run of equal labels among a warp's rows
-# of a 128-token tile (at most 19 tokens) in fp32 and adds the run sums to
-# fp32 accumulators with atomics, in no fixed order. With R <= n runs for a
-# cluster of n members, recursive fp32 summation bounds the error of its sum
-# by (R - 1 + 18) 2^-24 sum|x| <= (n + 17) 2^-24 sum|x|, and the oracle's flush
-# of components below 2^-24 moves it by at most 2^-24 per member: the mean is
-# within (n + 18) 2^-24 mean|x| + 2^-24 of the oracle's exact mean, and the
-# two fp32 roundings can part by one more unit in the last place.
-CENT_ABS = 2.0 ** -24
+# Centroid update: the member sums are exact on both sides (the oracle sums in
+# fp64 in token order, the GPU adds fp64 partial sums in any order; with the
+# components below 2^-24 counted as zero every partial sum is a multiple of
+# 2^-31 below 2^22, which fp64 holds exactly), and both round sum / n once to
+# fp32: given the same labels the centroids are bit-identical.
 
 
 def check_centroids(gpu_cent, x_bits, labels, want, old, what=""):
-    """GPU centroids against the oracle's update (want) for the same labels;
-    clusters left empty must keep their old centroid exactly."""
-    xf = np.abs(bf16_bits_to_f32(x_bits).astype(np.float64))
+    """GPU centroids against the oracle's update (want) for the same labels:
+    bit-identical, and clusters left empty keep their old centroid exactly."""
     C = want.shape[0]
     n = np.bincount(labels, minlength=C)
-    absum = np.zeros(want.shape, np.float64)
-    np.add.at(absum, labels, xf)
-    mean_abs = absum / np.maximum(n, 1)[:, None]
-    tol = (n[:, None] + 18) * 2.0 ** -24 * mean_abs + CENT_ABS + \
-        np.spacing(np.abs(want).astype(np.float32)).astype(np.float64)
-    err = np.abs(gpu_cent.astype(np.float64) - want.astype(np.float64))
     empty = n == 0
     assert np.array_equal(gpu_cent[empty].view(np.uint32), old[empty].view(np.uint32)), what
-    bad = (err > tol) & ~empty[:, None]
-    assert not bad.any(), f"{what}: {int(bad.sum())} centroid components beyond the bound, " \
-                          f"worst {float((err - tol).max()):.3e}"
+    diff = gpu_cent.view(np.uint32) != want.astype(np.float32).view(np.uint32)
+    assert not diff.any(), f"{what}: {int(diff.sum())} centroid components differ from the oracle's, " \
+                           f"largest gap {float(np.abs(gpu_cent.astype(np.float64) - want)[diff].max()):.3e}"
 
 
 def oracle_plan_heads(w: workload.Workload, q, k, heads, keeps, iters=None, mode=0):

@@ -7,8 +7,7 @@ another GPU stage) and its outputs are compared with the oracle's:
   trajectory (the GPU step started from the oracle's exact state): labels
   agree on >= 99.9% of tokens and every disagreement sits where the oracle's
   own fp64 distances are within 1e-4 (relative); with full agreement the
-  sizes are exact and every centroid lies within the bound of its fp32 member
-  sums, (n + 18) 2^-24 mean|x| + 2^-24 + 1 ulp of the oracle's;
+  sizes are exact and the centroids bit-identical (both sides sum exactly);
 * whole clustering run on the GPU alone: a drift report against the oracle's
   run (>= 98%; the trajectories may part at a near-tie);
 * mask + tail merge, permutation, query tiles, gathered copies: bit-exact;
@@ -139,8 +138,8 @@ def test_cluster_trajectory(name):
     """Hard gate along the oracle's whole k-means trajectory: at every half-step
     of every round the GPU step, started from the oracle's exact state, agrees
     with the oracle's step (>= 99.9%, disagreements only at relative distance
-    gaps < 1e-4; when all labels agree, exact sizes and centroids within the
-    bound of check_centroids)."""
+    gaps < 1e-4; when all labels agree, exact sizes and bit-identical
+    centroids)."""
     w = SMALL[name]
     q, k, _ = workload.make_qkv(w)
     qd, kd, _ = qkv_tensors(q, k, k, w.B, w.H)
