@@ -1,5 +1,11 @@
 """Builds libsvoo.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
+It also links libsvoo_stall.so, a test-only variant whose pipelined kernels
+(attention, clustering assignment) are compiled with SVOO_TEST_STALL: one
+pipeline wait on a barrier that nothing completes and a pipeline wait budget
+of about 10 ms, so a test can drive the device timeout path and read the
+error word. No product code loads it.
+
     python -m free_sparse_attention_head_b200.build [--force]
 """
 from __future__ import annotations
@@ -7,12 +13,15 @@ from __future__ import annotations
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsvoo.so")
+STALL_LIB = os.path.join(HERE, "libsvoo_stall.so")
 SOURCES = ["api.cu", "cluster.cu", "mask.cu", "permute.cu", "attn.cu", "psa.cu"]
+STALL_SOURCES = ["cluster.cu", "attn.cu"]  # the kernels with pipeline waits
 HEADERS = ["common.cuh", "internal.h"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
@@ -34,23 +43,39 @@ def _newest_input() -> float:
     return max(os.path.getmtime(p) for p in paths)
 
 
+def _link(out: str, objs) -> None:
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call([_nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
+                           "-o", tmp, *objs])
+    os.replace(tmp, out)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu to an object and link libsvoo.so; skipped when up to date."""
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_input():
+    """Compile every .cu to an object and link libsvoo.so (and the test-only
+    libsvoo_stall.so); skipped when both are up to date."""
+    newest = _newest_input()
+    if (not force and all(os.path.exists(p) and os.path.getmtime(p) >= newest
+                          for p in (LIB, STALL_LIB))):
         return LIB
     os.makedirs(BUILD, exist_ok=True)
-    objs = []
+    jobs = []  # (source, object, extra flags)
     for src in SOURCES:
-        obj = os.path.join(BUILD, src.replace(".cu", ".o"))
-        cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o", obj]
+        jobs.append((src, os.path.join(BUILD, src.replace(".cu", ".o")), []))
+    for src in STALL_SOURCES:
+        jobs.append((src, os.path.join(BUILD, src.replace(".cu", "_stall.o")), ["-DSVOO_TEST_STALL"]))
+
+    def compile_one(job):
+        src, obj, extra = job
+        cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
-        objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call([_nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
-                           "-o", tmp, *objs])
-    os.replace(tmp, LIB)
+
+    with ThreadPoolExecutor(max_workers=min(len(jobs), os.cpu_count() or 1)) as ex:
+        list(ex.map(compile_one, jobs))
+    _link(LIB, [os.path.join(BUILD, src.replace(".cu", ".o")) for src in SOURCES])
+    _link(STALL_LIB, [os.path.join(BUILD, src.replace(".cu", "_stall.o") if src in STALL_SOURCES
+                                   else src.replace(".cu", ".o")) for src in SOURCES])
     return LIB
 
 

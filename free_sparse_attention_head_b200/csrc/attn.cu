@@ -50,6 +50,9 @@ struct AttnSmem {
   uint64_t k_full[2], v_full[2], k_empty[2], v_empty[2];
   uint64_t s_full[2], p_half[2], p_full[2];
   uint64_t o_done, mma_final;
+#ifdef SVOO_TEST_STALL
+  uint64_t stall;  // test-only: a barrier that nothing completes
+#endif
   uint32_t tmem_base;
   int abort;
   int ncl;      // kept key groups with at least one row
@@ -149,6 +152,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     mbar_init(smem_u32(&S->o_done), 1);
     mbar_init(smem_u32(&S->mma_final), 1);
+#ifdef SVOO_TEST_STALL
+    mbar_init(smem_u32(&S->stall), 1);
+#endif
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -213,11 +219,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   // registers: the producer / issuer warpgroup gives up what the softmax
   // warpgroups use (launch: 384 x 168 = 128 x kRegsLow + 256 x kRegsHigh);
   // each warpgroup's branch starts with its own setmaxnreg
+  int k_armed = -1, v_armed = -1;  // producer: last tile whose K / V load was issued
   if (warp < 4) {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   if (warp == 0 && nkv > 0) {
     // ---------------------------------------------------------------- producer
-    int k_armed = -1, v_armed = -1;  // last tile whose K / V load was issued
     if (lane == 0) {
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
@@ -255,16 +261,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     smem_u32(&S->v_full[st]), my_sub * 64, row);
       v_armed = j;
     }
-    if (*abort && lane == 0) {
-      // let every issued copy land before this CTA's shared memory is released
-      int dummy = 0;
-      for (int j = max(0, k_armed - 1); j <= k_armed; ++j)
-        mbar_wait(smem_u32(&S->k_full[j & 1]), (j >> 1) & 1, &dummy);
-      for (int j = max(0, v_armed - 1); j <= v_armed; ++j)
-        mbar_wait(smem_u32(&S->v_full[j & 1]), (j >> 1) & 1, &dummy);
-      dummy = 0;
-      mbar_wait(smem_u32(&S->q_full), 0, &dummy);
-    }
   } else if (warp == 1 && nkv > 0) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -272,6 +268,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t idesc_o = idesc_bf16_f32(kQRows, D, false, true);
       const int ntile = has_b ? 2 : 1;
       bool ok = mbar_wait(smem_u32(&S->q_full), 0, abort);
+#ifdef SVOO_TEST_STALL
+      ok = ok && mbar_wait(smem_u32(&S->stall), 0, abort);  // nothing completes it
+#endif
       for (int j = 0; j <= nkv && ok; ++j) {
         const int st = j & 1, pst = (j - 1) & 1;
         for (int t = 0; t < ntile && ok; ++t) {
@@ -313,8 +312,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       umma_commit(smem_u32(&S->o_done));
       // every MMA of this thread done before the TMEM is released
       umma_commit(smem_u32(&S->mma_final));
-      int dummy = 0;
-      mbar_wait(smem_u32(&S->mma_final), 0, &dummy);
+      mbar_wait_cleanup(smem_u32(&S->mma_final), 0);
     }
   }
   } else {
@@ -459,7 +457,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && *abort) report_error(err, kErrTimeoutAttn);
+  if (tid == 0 && *abort) {  // every role is done, so the flag is final here
+    report_error(err, kErrTimeoutAttn);
+    // let every copy the producer issued land before the shared memory goes
+    // away (only the last two of each ring can still be in flight)
+    if (nkv > 0) {
+      for (int j = max(0, k_armed - 1); j <= k_armed; ++j)
+        mbar_wait_cleanup(smem_u32(&S->k_full[j & 1]), (j >> 1) & 1);
+      for (int j = max(0, v_armed - 1); j <= v_armed; ++j)
+        mbar_wait_cleanup(smem_u32(&S->v_full[j & 1]), (j >> 1) & 1);
+      mbar_wait_cleanup(smem_u32(&S->q_full), 0);
+    }
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

@@ -6,15 +6,16 @@
 //
 // Kernels of one half-step (one side):
 //   metric_m_kernel   M from the other side's centroids and sizes (fp64)
-//   metric_nu_kernel  nu_j = M mu_j, kappa_j = mu_j . nu_j (fp64), |nu_j|, and
-//                     nu_j split into two bf16 rows (hi + lo)
-//   assign_kernel     persistent, warp-specialised, dynamically scheduled:
-//                     tcgen05 MMAs of 128-token tiles against [nu_hi | nu_lo]
-//                     into double-buffered TMEM; per token the score
-//                     kappa_j - 2 x.nu_j is bounded by the MMA error and a
-//                     token with a single candidate takes it
-//   fixup_kernel      the other tokens: candidates re-scored closer, then in
-//                     fp64 (ties to the smaller j)
+//   metric_nu_kernel  nu_j = M mu_j, kappa_j = mu_j . nu_j (fp64), |nu_j|,
+//                     nu_j split into two bf16 rows (hi + lo), -kappa_j/2 in
+//                     three bf16 parts, and per-block maxima for the bound
+//   assign_kernel     persistent, warp-specialised, dynamically scheduled
+//                     stream of 128-token tiles: tcgen05 MMAs against
+//                     [nu_hi | nu_lo | kappa] into double-buffered TMEM; per
+//                     token the score kappa_j - 2 x.nu_j is bounded by the
+//                     MMA error and a token with a single candidate takes it
+//   fixup_kernel      the other tokens, exactly in fp64: their listed
+//                     candidates, or every cluster (ties to the smaller j)
 //   update_kernel     member sums in fp64, exact (so order-independent), per
 //                     chunk of consecutive tokens grouped by label
 //   finalize_kernel   centroid = fp32(sum / count), empty clusters keep
@@ -156,14 +157,58 @@ __global__ void __launch_bounds__(kMThreads)
 }
 constexpr size_t kMetricMSmem = 2 * 2 * kMChunk * kMBlk * sizeof(double);  // 64 KB
 
+// Shared memory matrix descriptor without swizzle (K-major): 8-row x 16-byte
+// core matrices, `lbo` bytes between the two K halves of a 16-element row
+// chunk, `sbo` bytes between 8-row groups.
+__device__ __forceinline__ uint64_t plain_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;  // layout type 0: no swizzle
+}
+
+// byte offset of element (row, k) of a [rows][16] bf16 tile in that layout
+// (lbo = 128, sbo = 256)
+__host__ __device__ __forceinline__ uint32_t plain_offset(int row, int k) {
+  return static_cast<uint32_t>((row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+
+__device__ __forceinline__ uint16_t bf16_bits_rn(float f) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<const uint16_t*>(&b);
+}
+
+// -kappa/2 as three bf16 parts whose sum equals it to 2^-26 relative; a
+// padding column gets -2^114 and never wins
+__device__ __forceinline__ void kappa_parts(double kappa, bool real, uint16_t (&p)[3]) {
+  p[0] = p[1] = p[2] = 0;
+  if (!real) {
+    p[0] = 0xF880;
+    return;
+  }
+  const double v = -0.5 * kappa;
+  p[0] = bf16_bits_rn(static_cast<float>(v));
+  const double r1 = v - static_cast<double>(__uint_as_float(static_cast<uint32_t>(p[0]) << 16));
+  p[1] = bf16_bits_rn(static_cast<float>(r1));
+  const double r2 = r1 - static_cast<double>(__uint_as_float(static_cast<uint32_t>(p[1]) << 16));
+  p[2] = bf16_bits_rn(static_cast<float>(r2));
+}
+
 // nu_j = M mu_j and kappa_j = mu_j . nu_j in fp64; nu_j also as the pair of
 // bf16 rows nu_hi = bf16(nu_j), nu_lo = bf16(nu_j - nu_hi) that the scoring
 // MMA consumes (their sum is nu_j to 2^-18 relative), and |nu_j|. Clusters j
 // in [C, CP) are padding (nu = 0, kappa = +inf). grid (CP/32, BH), block 128:
 // warp w owns clusters j0 + 8w .. +7, lane owns dimensions 2 lane, 2 lane + 1
 // (and 64 + the same for d = 128). Rows of M arrive 16 at a time by cp.async,
-// one chunk ahead. M == nullptr means the identity.
+// one chunk ahead. M == nullptr means the identity. For the scoring MMA it
+// also writes, per head, the kappa parts tile (-kappa_j/2 in three bf16
+// parts, rows j of a [CP][16] tile in the no-swizzle core-matrix layout,
+// exactly as it lies in shared memory) and, per block of 32 clusters,
+// (max |nu_j|, max |kappa_j|) over its real clusters.
 constexpr int kNuRows = 16;
+constexpr int kExtraK = 16;  // K width of the kappa chunk of the scoring MMA
 constexpr int kNuMuStride = 130;  // doubles per staged centroid row (keeps 16-byte alignment)
 
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
@@ -177,8 +222,10 @@ __global__ void __launch_bounds__(128)
     metric_nu_kernel(const double* __restrict__ M, const float* __restrict__ cent, int C, int CP,
                      int d, double* __restrict__ nu64, uint16_t* __restrict__ nu_hi,
                      uint16_t* __restrict__ nu_lo, double* __restrict__ kappa64,
-                     float* __restrict__ kappa32, float* __restrict__ nunorm) {
+                     float* __restrict__ kappa32, float* __restrict__ nunorm, uint16_t* __restrict__ kimg,
+                     float2* __restrict__ numax) {
   extern __shared__ __align__(16) double nsm[];
+  __shared__ float2 wmax[4];
   double* mu = nsm;                          // [32][kNuMuStride]
   double* mch = mu + 32 * kNuMuStride;       // two buffers of [16][d]
   const int h = blockIdx.y, j0 = blockIdx.x * 32;
@@ -238,6 +285,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
       for (int v = 0; v < 4; ++v) acc[u][v] = v < nd ? mw[u * kNuMuStride + dim[v]] : 0.0;
   }
+  float mx_n = 0.f, mx_k = 0.f;
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int j = j0 + 8 * warp + u;
@@ -275,24 +323,50 @@ __global__ void __launch_bounds__(128)
       k2 += __shfl_xor_sync(0xffffffffu, k2, o);
     }
     if (lane == 0) {
+      const float nn = j < C ? static_cast<float>(sqrt(k2)) : 0.f;
       kappa64[h * CP + j] = j < C ? k1 : INFINITY;
       kappa32[h * CP + j] = j < C ? static_cast<float>(k1) : INFINITY;
-      nunorm[h * CP + j] = j < C ? static_cast<float>(sqrt(k2)) : 0.f;
+      nunorm[h * CP + j] = nn;
+      uint16_t p[3];
+      kappa_parts(k1, j < C, p);
+      uint8_t* img = reinterpret_cast<uint8_t*>(kimg + static_cast<size_t>(h) * CP * kExtraK);
+      *reinterpret_cast<uint4*>(img + plain_offset(j, 0)) =
+          make_uint4(p[0] | (static_cast<uint32_t>(p[1]) << 16), p[2], 0u, 0u);
+      *reinterpret_cast<uint4*>(img + plain_offset(j, 8)) = make_uint4(0u, 0u, 0u, 0u);
+      if (j < C) {
+        mx_n = fmaxf(mx_n, nn);
+        mx_k = fmaxf(mx_k, static_cast<float>(fabs(k1)));
+      }
     }
+  }
+  if (lane == 0) wmax[warp] = make_float2(mx_n, mx_k);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float2 m = wmax[0];
+    for (int w = 1; w < 4; ++w) m = make_float2(fmaxf(m.x, wmax[w].x), fmaxf(m.y, wmax[w].y));
+    numax[h * (CP / 32) + blockIdx.x] = m;
   }
 }
 inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d) * sizeof(double); }
 
 // ---------------------------------------------------------------- assign
 //
-// Persistent, warp-specialised kernel, one CTA per SM. The (head, 128-token
-// tile) space is handed out in chunks of kChunkTiles tiles of one head through
-// per-head counters: a CTA starts at its own head and moves on to the next
-// head with chunks left, so SMs that run this kernel faster take more chunks
-// (on B200 some SMs ran the same tiles up to 1.5x slower than others, so a
-// static split left the fast ones idle). Tile i of a CTA uses X buffer i % 2
-// in shared memory and TMEM accumulator i % 2 (CP fp32 columns).
-//   producer (warp 0)   TMA of the X tile, then one tcgen05 chain per tile:
+// Persistent, warp-specialised kernel, one CTA per SM, over a stream of
+// 128-token tiles. The (head, tile) space is handed out in chunks of
+// kChunkTiles tiles of one head through per-head counters: a CTA starts at its
+// own head and moves on to the next head with chunks left, so SMs that run
+// this kernel faster take more chunks (on B200 some SMs ran the same tiles up
+// to 1.5x slower than others, so a static split left the fast ones idle).
+// Tile i of a CTA uses X buffer i % 2 and TMEM accumulator i % 2 (CP fp32
+// columns).
+//   scheduler (warp 17) claims the CTA's next chunk while the current one
+//                       runs (one chunk ahead); its lanes probe 32 head
+//                       counters at a time.
+//   producer (warp 0)   streams the chunks' tiles: TMA of the X tile, whose
+//                       head and tile index go into shared memory beside it;
+//                       on a head change, once the tensor cores are done with
+//                       the old head, TMA of the new head's nu_hi, nu_lo and
+//                       kappa parts; then one tcgen05 chain per tile:
 //                       u = X . nu_hi^T + X . nu_lo^T + 1 . (-kappa/2)^T, the
 //                       last term a 16-wide K chunk of ones against -kappa_j/2
 //                       split into three bf16 parts, so u_j = x.nu_j - kappa_j/2
@@ -300,16 +374,19 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 //   scorers (warps 1-16) warp w reads TMEM lane quarter w % 4 (32 rows) and
 //                       column quarter (w - 1) / 4: each thread loads its row's
 //                       CP/4 scores into registers (then the accumulator goes
-//                       back), the quarter's maximum; the four quarters of a
-//                       row meet in shared memory for the row maximum U and
-//                       the error bound E; then each thread lists its
-//                       quarter's candidates u_j >= U - 2E (they contain the
-//                       exact argmin of the score). The quarter-0 warp of a
-//                       lane quarter decides its rows: one candidate is the
-//                       label; several go to the tile's deferred list (up to
-//                       kDeferSlots rows per 32 with up to kDeferCand
-//                       candidates each, label -1) or, beyond that, get label
-//                       -2 (all clusters); fixup_kernel decides them.
+//                       back) and takes the quarter's maximum; the four
+//                       quarters of a row meet in shared memory for the row
+//                       maximum U and the error bound E; each thread finds its
+//                       quarter's candidates u_j >= U - 2E (together they
+//                       contain the exact argmin of the score) and publishes
+//                       their count. From the four counts the four warps take
+//                       the same decision for the row: one candidate is the
+//                       label, written by the warp that holds it; several go
+//                       to the deferred list of the row's 32-row group (up to
+//                       kDeferSlots rows with up to kDeferCand candidates,
+//                       each warp writing its own); the rest (more candidates,
+//                       no free slot, or none at all) get label -2, every
+//                       cluster. fixup_kernel decides the listed and -2 rows.
 //
 // Error bound: nu_hi + nu_lo equals nu to 2^-18 relative and the three kappa
 // parts give kappa to 2^-26; the MMA's fp32 accumulation of 2d + 3 exact
@@ -323,19 +400,16 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 constexpr int kXnormCompute = 0, kXnormStore = 1, kXnormLoad = 2;
 
 constexpr int kScorerWarps = 16;
-constexpr int kAssignWarps = 1 + kScorerWarps;
+constexpr int kSchedWarp = 1 + kScorerWarps;
+constexpr int kAssignWarps = 2 + kScorerWarps;
 constexpr int kAssignThreads = kAssignWarps * 32;
-constexpr int kScorers = kScorerWarps * 32;
 constexpr int kTileRows = 128;
-constexpr int kQuarterCand = 4;      // candidates kept per column quarter
+constexpr int kQuarterCand = 4;      // candidates a quarter may add to a listed row
 constexpr int kDeferSlots = 8;       // listed deferred rows per 32 rows of a tile
 constexpr int kDeferCand = 8;        // candidates of a listed deferred row
 constexpr int kDeferAll = 1 << 8;    // defer_count flag: some rows of the group have label -2
-constexpr int kChunkTiles = 16;      // tiles per claimed chunk
-constexpr int kAssignHeader = 12288; // AssignSmem, keeps the X buffers 1024-aligned
-constexpr int kExtraK = 16;          // the kappa chunk of the MMA
-// named barriers: 1..4 the four scorer warps of a TMEM lane quarter, 5 all scorers
-constexpr int kBarScorers = 5;
+constexpr int kChunkTiles = 4;       // tiles per claimed chunk
+constexpr int kAssignHeader = 6144;  // AssignSmem, keeps the X buffers 1024-aligned
 
 // A row with several candidates, decided by fixup_kernel.
 struct DeferRec {
@@ -346,15 +420,17 @@ struct DeferRec {
 
 struct AssignSmem {
   uint64_t x_full[2], x_free[2], t_full[2], t_free[2];
+  uint64_t nu_full, sched_full, sched_free;
+#ifdef SVOO_TEST_STALL
+  uint64_t stall;  // test-only: a barrier that nothing completes
+#endif
   uint32_t tmem_base;
   int abort;
-  int claim_h, claim_c;
-  float max_nrm;
-  float max_kap;
-  float xq[4][kTileRows];                  // |x|^2 per column quarter's dimensions
-  float mq[4][kTileRows];                  // per-quarter maxima of u
-  uint8_t kc[4][kTileRows];                // candidates per quarter (saturating)
-  int16_t cand[4][kTileRows][kQuarterCand];
+  int tile_h[2], tile_t[2];  // head and tile of each X buffer's tile (head -1: the end)
+  int sched_h, sched_c;      // the scheduler's claimed chunk (head -1: none left)
+  float xq[4][kTileRows];    // |x|^2 per column quarter's dimensions
+  float mq[4][kTileRows];    // per-quarter maxima of u
+  uint32_t kc[kTileRows];    // candidates per column quarter, a byte each (saturating)
 };
 static_assert(sizeof(AssignSmem) <= kAssignHeader, "assign header overflow");
 
@@ -376,44 +452,41 @@ __device__ __forceinline__ int named_sync_or(int id, int threads, int flag) {
   return r;
 }
 
-// Shared memory matrix descriptor without swizzle (K-major): 8-row x 16-byte
-// core matrices, `lbo` bytes between the two K halves of a 16-element row
-// chunk, `sbo` bytes between 8-row groups.
-__device__ __forceinline__ uint64_t plain_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
-  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
-  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  return d;  // layout type 0: no swizzle
+// untiled bulk copy global -> shared, completing on `bar` (bytes; 16-byte
+// aligned addresses and size)
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
-// byte offset of element (row, k) of a [rows][16] bf16 tile in that layout
-// (lbo = 128, sbo = 256)
-__device__ __forceinline__ uint32_t plain_offset(int row, int k) {
-  return static_cast<uint32_t>((row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
-}
-
-__device__ __forceinline__ uint16_t bf16_bits_rn(float f) {
-  const __nv_bfloat16 b = __float2bfloat16_rn(f);
-  return *reinterpret_cast<const uint16_t*>(&b);
+// bit (q) of m set where v >= thr: a compare and a predicated OR per value
+__device__ __forceinline__ void mark_ge(uint32_t& m, float v, float thr, uint32_t bit) {
+  asm("{\n\t.reg .pred p;\n\t"
+      "setp.ge.f32 p, %1, %2;\n\t"
+      "@p or.b32 %0, %0, %3;\n\t}"
+      : "+r"(m)
+      : "f"(v), "f"(thr), "r"(bit));
 }
 
 // grid: min(#SMs, chunks) CTAs, block kAssignThreads. Dynamic smem:
 // [AssignSmem][X 2 x 128 x D bf16][nu_hi CP x D][nu_lo CP x D][ones 128 x 16][kappa parts CP x 16]
+// kimg: per head the kappa parts tile as it lies in shared memory; numax: per
+// head and 32-cluster block, (max |nu_j|, max |kappa_j|).
 template <int D, int CP>
 __global__ void __launch_bounds__(kAssignThreads, 1)
-    assign_kernel(const __grid_constant__ CUtensorMap xmap, int N, int nv, int C, int BH,
-                  const uint16_t* __restrict__ nu_hi, const uint16_t* __restrict__ nu_lo,
-                  const double* __restrict__ kappa64, const float* __restrict__ nunorm,
+    assign_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap himap,
+                  const __grid_constant__ CUtensorMap lomap, int N, int nv, int C, int BH,
+                  const uint16_t* __restrict__ kimg, const float2* __restrict__ numax,
                   int32_t* __restrict__ head_next, int32_t* __restrict__ assign,
                   int32_t* __restrict__ defer_count, DeferRec* __restrict__ defer,
-                  float* __restrict__ xnorm, int xnorm_mode, float* __restrict__ head_max,
-                  int* __restrict__ err) {
+                  float* __restrict__ xnorm, int xnorm_mode, int* __restrict__ err) {
   constexpr int kQCols = CP / 4;      // score columns per scorer thread
   constexpr int kLoads = kQCols / 32;  // 32-column TMEM loads per thread
   constexpr uint32_t kXBytes = kTileRows * D * 2;
   constexpr uint32_t kNuBytes = CP * D * 2;
+  constexpr uint32_t kKBytes = CP * kExtraK * 2;
   static_assert(CP == 128 || CP == 256, "CP must be 128 or 256");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -439,8 +512,16 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       mbar_init(smem_u32(&S->t_full[b]), 1);
       mbar_init(smem_u32(&S->t_free[b]), kScorerWarps);
     }
+    mbar_init(smem_u32(&S->nu_full), 1);
+    mbar_init(smem_u32(&S->sched_full), 1);
+    mbar_init(smem_u32(&S->sched_free), 1);
+#ifdef SVOO_TEST_STALL
+    mbar_init(smem_u32(&S->stall), 1);
+#endif
     fence_mbar_init();
     tma_prefetch_desc(&xmap);
+    tma_prefetch_desc(&himap);
+    tma_prefetch_desc(&lomap);
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(&S->tmem_base), 2 * CP);
@@ -451,6 +532,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const int row = e / kExtraK, k = e % kExtraK;
     *reinterpret_cast<uint16_t*>(ones + plain_offset(row, k)) = k < 3 ? 0x3F80 : 0;
   }
+  fence_proxy_async_smem();  // read by the tensor cores
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -458,146 +540,190 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   volatile int* abort = &S->abort;
   constexpr uint32_t idesc = idesc_bf16_f32(128, CP, false, false);
 
-  // producer state (warp 0, lane 0)
-  uint32_t tma_pend = 0;         // buffers with a TMA not yet waited on
+  // producer state (warp 0, lane 0), also read by the abort path below
+  uint32_t tma_pend = 0;         // X buffers with a TMA not yet waited on
   uint32_t tma_par[2] = {0, 0};  // x_full parity each of them completes
   int mma_last = -1;
+  bool nu_pend = false;          // operand copy not yet waited on
+  uint32_t nu_par = 0;           // nu_full parity of the next operand copy
 
-  int i = 0;  // tiles started by this CTA: selects buffers and barrier phases
-  int cur_h = -1;
-  int h_from = static_cast<int>(static_cast<long long>(blockIdx.x) * BH / gridDim.x);
-  while (true) {
-    if (tid == 0) {  // claim the next chunk: this head first, then the following ones
+  if (warp == kSchedWarp) {
+    // ------------------------------------------------------------ scheduler
+    int h_from = static_cast<int>(static_cast<long long>(blockIdx.x) * BH / gridDim.x);
+    for (int n = 0;; ++n) {
+      int ok = 1;
+      if (lane == 0 && n >= 1) ok = mbar_wait(smem_u32(&S->sched_free), (n - 1) & 1, abort) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       int found = -1, c = 0;
-      for (int k = 0; k < BH && found < 0; ++k) {
+      // heads h_from, h_from + 1, ... (cyclically), 32 at a time; a head whose
+      // counter has run out stays so, so every try that fails ends a head
+      for (int k0 = 0; k0 < BH && found < 0; k0 += 32) {
+        const int k = k0 + lane;
         const int hh = h_from + k < BH ? h_from + k : h_from + k - BH;
-        const int got = atomicAdd(&head_next[hh], 1);
-        if (got < nchunk) {
-          found = hh;
-          c = got;
+        const int open = (k < BH && *reinterpret_cast<volatile int32_t*>(head_next + hh) < nchunk) ? 1 : 0;
+        unsigned m = __ballot_sync(0xffffffffu, open);
+        while (m && found < 0) {
+          const int l = __ffs(m) - 1;
+          m &= m - 1;
+          int got = 0;
+          if (lane == l) got = atomicAdd(&head_next[hh], 1);
+          got = __shfl_sync(0xffffffffu, got, l);
+          const int hl = __shfl_sync(0xffffffffu, hh, l);
+          if (got < nchunk) {
+            found = hl;
+            c = got;
+          }
         }
       }
-      S->claim_h = found;
-      S->claim_c = c;
-    }
-    __syncthreads();  // every role is done with the previous chunk
-    if (__syncthreads_or(S->claim_h < 0 || *abort)) break;
-    const int h = S->claim_h;
-    const int t0 = S->claim_c * kChunkTiles, t1 = min(ntiles, t0 + kChunkTiles);
-    h_from = h;
-    const int row0 = h * N;
-    if (h != cur_h) {  // head h: nu_hi, nu_lo into the swizzled K-major layout of the B operand,
-                       // -kappa/2 in three bf16 parts into the kappa chunk, and the bound's maxima
-      constexpr int chunks = D / 8;
-      const uint4* srch = reinterpret_cast<const uint4*>(nu_hi + static_cast<size_t>(h) * CP * D);
-      const uint4* srcl = reinterpret_cast<const uint4*>(nu_lo + static_cast<size_t>(h) * CP * D);
-      for (int e = tid; e < CP * chunks; e += kAssignThreads) {
-        const int j = e / chunks, c = e % chunks;
-        const uint32_t off = sw128_offset(j, c * 8, CP);
-        const uint4 vh = __ldg(srch + e), vl = __ldg(srcl + e);
-        *reinterpret_cast<uint4*>(nuh + off) = vh;
-        *reinterpret_cast<uint4*>(nul + off) = vl;
-      }
-      for (int j = tid; j < CP; j += kAssignThreads) {
-        uint16_t p[3] = {0, 0, 0};
-        if (j < C) {
-          const double v = -0.5 * kappa64[h * CP + j];
-          p[0] = bf16_bits_rn(static_cast<float>(v));
-          const double r1 = v - static_cast<double>(__uint_as_float(static_cast<uint32_t>(p[0]) << 16));
-          p[1] = bf16_bits_rn(static_cast<float>(r1));
-          const double r2 = r1 - static_cast<double>(__uint_as_float(static_cast<uint32_t>(p[1]) << 16));
-          p[2] = bf16_bits_rn(static_cast<float>(r2));
-        } else {
-          p[0] = 0xF880;  // -2^114: a padding column never wins
-        }
-        for (int k = 0; k < kExtraK; ++k)
-          *reinterpret_cast<uint16_t*>(kparts + plain_offset(j, k)) = k < 3 ? p[k] : 0;
-      }
-      if (warp == 0) {
-        float mn = 0.f, mk = 0.f;
-        for (int j = lane; j < C; j += 32) {
-          mn = fmaxf(mn, nunorm[h * CP + j]);
-          mk = fmaxf(mk, static_cast<float>(fabs(kappa64[h * CP + j])));
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          mn = fmaxf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-          mk = fmaxf(mk, __shfl_xor_sync(0xffffffffu, mk, o));
-        }
-        if (lane == 0) {
-          S->max_nrm = mn;
-          S->max_kap = mk;
-          head_max[2 * h] = mn;  // for fixup_kernel (every CTA of the head writes the same)
-          head_max[2 * h + 1] = mk;
-        }
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-      cur_h = h;
-    }
-
-    if (warp == 0) {
-      // ------------------------------------------------------------ producer
+      if (found >= 0) h_from = found;
       if (lane == 0) {
-        auto issue_tma = [&](int ii, int tt) -> bool {
-          const int b = ii & 1;
-          if (ii >= 2 && !mbar_wait(smem_u32(&S->x_free[b]), ((ii >> 1) - 1) & 1, abort)) return false;
-          mbar_arrive_expect_tx(smem_u32(&S->x_full[b]), kXBytes);
-          for (int s = 0; s < D / 64; ++s)
-            tma_load_2d(&xmap, smem_u32(xs + b * kXBytes + s * kTileRows * 128), smem_u32(&S->x_full[b]),
-                        s * 64, row0 + tt * kTileRows);
-          tma_pend |= 1u << b;
-          tma_par[b] = (ii >> 1) & 1;
-          return true;
-        };
-        bool ok = issue_tma(i, t0);
-        const uint32_t ha = smem_u32(nuh), la = smem_u32(nul);
-        const uint64_t ad_k = plain_desc(smem_u32(ones), 128, 256);
-        const uint64_t bd_k = plain_desc(smem_u32(kparts), 128, 256);
-        for (int tt = t0; ok && tt < t1; ++tt) {
-          const int ii = i + (tt - t0), b = ii & 1;
-          if (tt + 1 < t1 && !issue_tma(ii + 1, tt + 1)) break;
-          if (!mbar_wait(smem_u32(&S->x_full[b]), (ii >> 1) & 1, abort)) break;
-          tma_pend &= ~(1u << b);
-          if (ii >= 2 && !mbar_wait(smem_u32(&S->t_free[b]), ((ii >> 1) - 1) & 1, abort)) break;
-          tc_fence_after();
-          const uint32_t dt = tmem + b * CP;
-          const uint32_t xa = smem_u32(xs + b * kXBytes);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int sub = kk >> 2, off = (kk & 3) * 32;
-            umma_f16(dt, sw128_desc(xa + sub * kTileRows * 128 + off, 16, 1024),
-                     sw128_desc(ha + sub * CP * 128 + off, 16, 1024), idesc, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const int sub = kk >> 2, off = (kk & 3) * 32;
-            umma_f16(dt, sw128_desc(xa + sub * kTileRows * 128 + off, 16, 1024),
-                     sw128_desc(la + sub * CP * 128 + off, 16, 1024), idesc, 1);
-          }
-          umma_f16(dt, ad_k, bd_k, idesc, 1);
-          umma_commit(smem_u32(&S->t_full[b]));
-          mma_last = ii;
-        }
+        S->sched_h = found;
+        S->sched_c = c;
+        mbar_arrive(smem_u32(&S->sched_full));
       }
-      __syncwarp();
-    } else {
-      // ------------------------------------------------------------ scorers
-      const int lq = warp & 3;          // TMEM lane quarter
-      const int cq = (warp - 1) >> 2;   // column quarter
-      const int r = lq * 32 + lane;     // tile row
-      const int quad_bar = 1 + lq;
-      const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
-      const float max_nrm = S->max_nrm, max_kap = S->max_kap;
-      for (int tt = t0; tt < t1; ++tt) {
-        const int ii = i + (tt - t0), b = ii & 1;
-        const uint32_t ph = (ii >> 1) & 1;
-        // the MMA of this tile (and so its X copy) is complete
-        const int late = (mbar_wait(smem_u32(&S->t_full[b]), ph, abort) &&
-                          mbar_wait(smem_u32(&S->x_full[b]), ph, abort)) ? 0 : 1;
-        if (named_sync_or(kBarScorers, kScorers, late)) break;  // every scorer leaves together
+      if (found < 0) break;
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int n_pop = 0, ch = -1, ct = 0, ce = 0;  // current chunk: head, next tile, end
+      // the next tile of the stream: 1 a tile, 0 the end, -1 a timeout
+      auto next_tile = [&](int& h, int& tt) -> int {
+        if (ct >= ce) {
+          if (!mbar_wait(smem_u32(&S->sched_full), n_pop & 1, abort)) return -1;
+          ch = S->sched_h;
+          const int c = S->sched_c;
+          mbar_arrive(smem_u32(&S->sched_free));
+          ++n_pop;
+          if (ch < 0) return 0;
+          ct = c * kChunkTiles;
+          ce = min(ntiles, ct + kChunkTiles);
+        }
+        h = ch;
+        tt = ct++;
+        return 1;
+      };
+      // X tile ii (head -1: the end of the stream, which completes the slot's
+      // x_full without a copy; t_full only ever completes by an MMA commit, so
+      // a wait for a given tile's MMA cannot be completed by this marker)
+      auto issue_tma = [&](int ii, int h, int tt) -> bool {
+        const int b = ii & 1;
+        if (ii >= 2 && !mbar_wait(smem_u32(&S->x_free[b]), ((ii >> 1) - 1) & 1, abort)) return false;
+        S->tile_h[b] = h;
+        S->tile_t[b] = tt;
+        if (h < 0) {
+          mbar_arrive(smem_u32(&S->x_full[b]));
+          return true;
+        }
+        mbar_arrive_expect_tx(smem_u32(&S->x_full[b]), kXBytes);
+        for (int s = 0; s < D / 64; ++s)
+          tma_load_2d(&xmap, smem_u32(xs + b * kXBytes + s * kTileRows * 128), smem_u32(&S->x_full[b]),
+                      s * 64, h * N + tt * kTileRows);
+        tma_pend |= 1u << b;
+        tma_par[b] = (ii >> 1) & 1;
+        return true;
+      };
+      // head h's MMA operands, once the tensor cores are done with the old ones
+      auto load_nu = [&](int h) -> bool {
+        if (mma_last >= 0 && !mbar_wait(smem_u32(&S->t_full[mma_last & 1]), (mma_last >> 1) & 1, abort))
+          return false;
+        mbar_arrive_expect_tx(smem_u32(&S->nu_full), 2 * kNuBytes + kKBytes);
+        for (int s = 0; s < D / 64; ++s) {
+          tma_load_2d(&himap, smem_u32(nuh + s * CP * 128), smem_u32(&S->nu_full), s * 64, h * CP);
+          tma_load_2d(&lomap, smem_u32(nul + s * CP * 128), smem_u32(&S->nu_full), s * 64, h * CP);
+        }
+        bulk_load(smem_u32(kparts), kimg + static_cast<size_t>(h) * CP * kExtraK, kKBytes,
+                  smem_u32(&S->nu_full));
+        nu_pend = true;
+        if (!mbar_wait(smem_u32(&S->nu_full), nu_par, abort)) return false;
+        nu_pend = false;
+        nu_par ^= 1u;
+        return true;
+      };
+      const uint32_t ha = smem_u32(nuh), la = smem_u32(nul);
+      const uint64_t ad_k = plain_desc(smem_u32(ones), 128, 256);
+      const uint64_t bd_k = plain_desc(smem_u32(kparts), 128, 256);
+      int hA = -1, tA = 0, loaded_h = -1;
+#ifdef SVOO_TEST_STALL
+      const bool go = mbar_wait(smem_u32(&S->stall), 0, abort);  // nothing completes it
+#else
+      constexpr bool go = true;
+#endif
+      int st = go ? next_tile(hA, tA) : -1;
+      bool ok = st >= 0 && issue_tma(0, st == 1 ? hA : -1, tA);
+      for (int ii = 0; ok && st == 1; ++ii) {
+        int hB = -1, tB = 0;
+        const int st2 = next_tile(hB, tB);
+        if (st2 < 0 || !issue_tma(ii + 1, st2 == 1 ? hB : -1, tB)) break;
+        const int b = ii & 1;
+        if (!mbar_wait(smem_u32(&S->x_full[b]), (ii >> 1) & 1, abort)) break;
+        tma_pend &= ~(1u << b);
+        if (ii >= 2 && !mbar_wait(smem_u32(&S->t_free[b]), ((ii >> 1) - 1) & 1, abort)) break;
+        if (hA != loaded_h) {
+          if (!load_nu(hA)) break;
+          loaded_h = hA;
+        }
         tc_fence_after();
-        const int tok = tt * kTileRows + r;
-        float xsq = 0.f;
+        const uint32_t dt = tmem + b * CP;
+        const uint32_t xa = smem_u32(xs + b * kXBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int sub = kk >> 2, off = (kk & 3) * 32;
+          umma_f16(dt, sw128_desc(xa + sub * kTileRows * 128 + off, 16, 1024),
+                   sw128_desc(ha + sub * CP * 128 + off, 16, 1024), idesc, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int sub = kk >> 2, off = (kk & 3) * 32;
+          umma_f16(dt, sw128_desc(xa + sub * kTileRows * 128 + off, 16, 1024),
+                   sw128_desc(la + sub * CP * 128 + off, 16, 1024), idesc, 1);
+        }
+        umma_f16(dt, ad_k, bd_k, idesc, 1);
+        umma_commit(smem_u32(&S->t_full[b]));
+        mma_last = ii;
+        hA = hB;
+        tA = tB;
+        st = st2;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ scorers
+    const int lq = warp & 3;          // TMEM lane quarter
+    const int cq = (warp - 1) >> 2;   // column quarter
+    const int r = lq * 32 + lane;     // tile row
+    const int quad_bar = 1 + lq;      // named barrier of the lane quarter's four warps
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
+    const unsigned lanes_below = (1u << lane) - 1u;
+    int cur_h = -1;
+    float max_nrm = 0.f, max_kap = 0.f;
+    for (int ii = 0;; ++ii) {
+      const int b = ii & 1;
+      const uint32_t ph = (ii >> 1) & 1;
+      // the slot's X copy (or the end-of-stream marker) is there, then, for a
+      // real tile, its MMA is complete
+      bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S->x_full[b]), ph, abort));
+      const int h = ok ? S->tile_h[b] : -1;
+      const int tt = ok ? S->tile_t[b] : 0;
+      if (ok && h >= 0) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S->t_full[b]), ph, abort));
+      const bool done = !ok || h < 0;  // a timeout, or the end of the stream
+      const int tok = tt * kTileRows + r;
+      float xsq = 0.f;
+      float v[kQCols];
+      if (!done) {
+        tc_fence_after();
+        if (h != cur_h) {  // the head's bound maxima
+          float mn = 0.f, mk = 0.f;
+#pragma unroll
+          for (int p = 0; p < CP / 32; ++p) {
+            const float2 m = __ldg(numax + h * (CP / 32) + p);
+            mn = fmaxf(mn, m.x);
+            mk = fmaxf(mk, m.y);
+          }
+          max_nrm = mn;
+          max_kap = mk;
+          cur_h = h;
+        }
         if (xnorm_mode == kXnormLoad) {
           // the scorers never read this X tile: it goes back to the producer at once
           __syncwarp();
@@ -608,11 +734,11 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
           for (int c = cq * (D / 4); c < (cq + 1) * (D / 4); c += 8) {
-            const uint4 v = *reinterpret_cast<const uint4*>(xb + sw128_offset(r, c, kTileRows));
-            const float f0 = __uint_as_float(v.x << 16), f1 = __uint_as_float(v.x & 0xffff0000u);
-            const float f2 = __uint_as_float(v.y << 16), f3 = __uint_as_float(v.y & 0xffff0000u);
-            const float f4 = __uint_as_float(v.z << 16), f5 = __uint_as_float(v.z & 0xffff0000u);
-            const float f6 = __uint_as_float(v.w << 16), f7 = __uint_as_float(v.w & 0xffff0000u);
+            const uint4 w = *reinterpret_cast<const uint4*>(xb + sw128_offset(r, c, kTileRows));
+            const float f0 = __uint_as_float(w.x << 16), f1 = __uint_as_float(w.x & 0xffff0000u);
+            const float f2 = __uint_as_float(w.y << 16), f3 = __uint_as_float(w.y & 0xffff0000u);
+            const float f4 = __uint_as_float(w.z << 16), f5 = __uint_as_float(w.z & 0xffff0000u);
+            const float f6 = __uint_as_float(w.w << 16), f7 = __uint_as_float(w.w & 0xffff0000u);
             a0 = fmaf(f0, f0, fmaf(f4, f4, a0));
             a1 = fmaf(f1, f1, fmaf(f5, f5, a1));
             a2 = fmaf(f2, f2, fmaf(f6, f6, a2));
@@ -624,7 +750,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         }
         // this quarter's scores into registers; then the accumulator is free
         const uint32_t ta = lane_base + b * CP + cq * kQCols;
-        float v[kQCols];
         tmem_ld32f(ta, v);
         if constexpr (kLoads == 2) tmem_ld32f(ta + 32, v + 32);
         tmem_wait_ld_f(v);
@@ -643,96 +768,82 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           }
         }
         S->mq[cq][r] = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-        named_sync(quad_bar, 128);
-        // candidates of this quarter within 2E of the row maximum
-        {
-          const float U = fmaxf(fmaxf(S->mq[0][r], S->mq[1][r]), fmaxf(S->mq[2][r], S->mq[3][r]));
-          if (xnorm_mode != kXnormLoad) {
-            xsq = (S->xq[0][r] + S->xq[1][r]) + (S->xq[2][r] + S->xq[3][r]);
-            if (xnorm_mode == kXnormStore && cq == 0 && tok < nv) xnorm[static_cast<size_t>(h) * nv + tok] = xsq;
-          }
-          const float thr = U - ldexpf(sqrtf(xsq) * max_nrm + 0.5f * max_kap, -12);
-          int k = 0;
-          int16_t cl[kQuarterCand] = {0, 0, 0, 0};
-#pragma unroll
-          for (int w32 = 0; w32 < kLoads; ++w32) {
-            // eight independent partial masks keep the OR chains short
-            uint32_t p8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) p8[u] = 0u;
-#pragma unroll
-            for (int q = 0; q < 32; ++q) p8[q & 7] |= (v[w32 * 32 + q] >= thr ? 1u : 0u) << q;
-            uint32_t bw = ((p8[0] | p8[1]) | (p8[2] | p8[3])) | ((p8[4] | p8[5]) | (p8[6] | p8[7]));
-            while (bw) {
-              const int q = __ffs(bw) - 1;
-              bw &= bw - 1;
-              if (k < kQuarterCand) cl[k] = static_cast<int16_t>(cq * kQCols + 32 * w32 + q);
-              ++k;
-            }
-          }
-          S->kc[cq][r] = static_cast<uint8_t>(min(k, 255));
-#pragma unroll
-          for (int q = 0; q < kQuarterCand; ++q) S->cand[cq][r][q] = cl[q];
-        }
-        named_sync(quad_bar, 128);
-        if (cq == 0) {  // the row's decision
-          int L = -3;   // not a video token
-          int total = 0;
-          bool listable = true;
-          if (tok < nv) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int kq = S->kc[q][r];
-              total += kq;
-              listable = listable && kq <= kQuarterCand;
-              // a padding column (only with non-finite input) is never listed
-              for (int u = 0; u < min(kq, kQuarterCand); ++u) listable = listable && S->cand[q][r][u] < C;
-            }
-            if (total == 1) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                if (S->kc[q][r] == 1) L = S->cand[q][r][0];
-              if (L >= C) L = -2;  // a padding column (only with non-finite input)
-            } else {
-              L = -1;
-            }
-          }
-          const size_t grp = (static_cast<size_t>(h) * ntiles + tt) * 4 + lq;
-          // listed rows get the slots in lane order; the rest are marked -2
-          const unsigned dm = __ballot_sync(0xffffffffu, L == -1 && listable && total <= kDeferCand);
-          const int slot = __popc(dm & ((1u << lane) - 1u));
-          if (L == -1) {
-            if (((dm >> lane) & 1u) && slot < kDeferSlots) {
-              DeferRec rec;
-              rec.tok = tok;
-              rec.n = total;
-              int n = 0;
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                for (int u = 0; u < S->kc[q][r]; ++u) rec.cand[n++] = S->cand[q][r][u];
-              for (; n < kDeferCand; ++n) rec.cand[n] = 0;
-              defer[grp * kDeferSlots + slot] = rec;
-            } else {
-              L = -2;  // too many to list: fixup_kernel compares every cluster
-            }
-          }
-          if (L != -3) assign[static_cast<size_t>(h) * nv + tok] = L;
-          // listed records (at most kDeferSlots), plus kDeferAll if any row has label -2
-          const unsigned all = __ballot_sync(0xffffffffu, L == -2);
-          if (lane == 0) defer_count[grp] = min(__popc(dm), kDeferSlots) | (all ? kDeferAll : 0);
-        }
       }
+      // the four warps of the lane quarter leave together
+      if (named_sync_or(quad_bar, 128, done ? 1 : 0)) break;
+      // candidates of this quarter within 2E of the row maximum
+      const float U = fmaxf(fmaxf(S->mq[0][r], S->mq[1][r]), fmaxf(S->mq[2][r], S->mq[3][r]));
+      if (xnorm_mode != kXnormLoad) {
+        xsq = (S->xq[0][r] + S->xq[1][r]) + (S->xq[2][r] + S->xq[3][r]);
+        if (xnorm_mode == kXnormStore && cq == 0 && tok < nv) xnorm[static_cast<size_t>(h) * nv + tok] = xsq;
+      }
+      const float thr = U - ldexpf(sqrtf(xsq) * max_nrm + 0.5f * max_kap, -12);
+      uint32_t mask[kLoads];
+#pragma unroll
+      for (int w32 = 0; w32 < kLoads; ++w32) {
+        uint32_t p8[8];  // eight partial masks keep the OR chains short
+#pragma unroll
+        for (int u = 0; u < 8; ++u) p8[u] = 0u;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) mark_ge(p8[q & 7], v[w32 * 32 + q], thr, 1u << q);
+        mask[w32] = ((p8[0] | p8[1]) | (p8[2] | p8[3])) | ((p8[4] | p8[5]) | (p8[6] | p8[7]));
+      }
+      uint64_t mm = mask[0];
+      if constexpr (kLoads == 2) mm |= static_cast<uint64_t>(mask[1]) << 32;
+      const int k = __popcll(mm);
+      reinterpret_cast<volatile uint8_t*>(&S->kc[r])[cq] = static_cast<uint8_t>(min(k, 255));
+      named_sync(quad_bar, 128);
+      // the row's decision, the same in the four warps
+      const uint32_t kw = S->kc[r];
+      const int k0 = kw & 255, k1 = (kw >> 8) & 255, k2 = (kw >> 16) & 255, k3 = kw >> 24;
+      const int total = (k0 + k1) + (k2 + k3);
+      const int kmax = max(max(k0, k1), max(k2, k3));
+      const int before = cq == 0 ? 0 : cq == 1 ? k0 : cq == 2 ? k0 + k1 : (k0 + k1) + k2;
+      const bool row = tok < nv;
+      const bool listable = row && total >= 2 && total <= kDeferCand && kmax <= kQuarterCand;
+      const unsigned dm = __ballot_sync(0xffffffffu, listable);
+      const int slot = __popc(dm & lanes_below);
+      const long long grp = (static_cast<long long>(h) * ntiles + tt) * 4 + lq;
+      int32_t* arow = assign + static_cast<size_t>(h) * nv + tok;
+      bool minus2 = false;
+      if (row && total == 1) {
+        if (k == 1) {  // the single candidate is this quarter's
+          const int j = cq * kQCols + (__ffsll(static_cast<long long>(mm)) - 1);
+          minus2 = j >= C;  // a padding column (only with non-finite input)
+          *arow = minus2 ? -2 : j;
+        }
+      } else if (listable && slot < kDeferSlots) {
+        DeferRec* dst = defer + grp * kDeferSlots + slot;
+        if (cq == 0) {
+          dst->tok = tok;
+          dst->n = total;
+        }
+#pragma unroll
+        for (int u = 0; u < kQuarterCand; ++u) {
+          if (u < k) {
+            const int q = __ffsll(static_cast<long long>(mm)) - 1;
+            mm &= mm - 1;
+            dst->cand[before + u] = static_cast<int16_t>(cq * kQCols + q);
+          }
+        }
+      } else if (row && cq == 0) {  // none, too many, or no free slot: every cluster
+        minus2 = true;
+        *arow = -2;
+      }
+      const unsigned any2 = __ballot_sync(0xffffffffu, minus2);
+      // word cq of the group: the listed rows (word 0) and kDeferAll
+      if (lane == 0)
+        defer_count[grp * 4 + cq] = (cq == 0 ? min(__popc(dm), kDeferSlots) : 0) | (any2 ? kDeferAll : 0);
     }
-    i += t1 - t0;
   }
   __syncthreads();
   if (*abort && tid == 0) {
     report_error(err, kErrTimeoutCluster);
     // copies and MMAs still in flight complete before the buffers go away
-    volatile int keep_waiting = 0;
     for (int b = 0; b < 2; ++b)
-      if (tma_pend & (1u << b)) mbar_wait(smem_u32(&S->x_full[b]), tma_par[b], &keep_waiting);
-    if (mma_last >= 0) mbar_wait(smem_u32(&S->t_full[mma_last & 1]), (mma_last >> 1) & 1, &keep_waiting);
+      if (tma_pend & (1u << b)) mbar_wait_cleanup(smem_u32(&S->x_full[b]), tma_par[b]);
+    if (nu_pend) mbar_wait_cleanup(smem_u32(&S->nu_full), nu_par);
+    if (mma_last >= 0) mbar_wait_cleanup(smem_u32(&S->t_full[mma_last & 1]), (mma_last >> 1) & 1);
   }
   tc_fence_before();
   __syncthreads();
@@ -741,107 +852,25 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 
 // ---------------------------------------------------------------- fixup
 //
-// Decides the rows the scorers could not: the listed deferred rows of every
-// (tile, 32-row group) and the rows labelled -2. One warp per group; lane l
-// holds dimensions (D/32) l .. (D/32) l + D/32 - 1 of the row. First, in fp32,
-// t_j = x.(nu_hi + nu_lo)_j - kappa_j / 2: the products are exact, and the
-// sums and the rounded -kappa_j/2 err by far less than
-// 2^-17 (|x||nu_j| + |kappa_j|), so every j within
-// E2 = 2^-16 (|x| max|nu| + max|kappa| / 2) of the best t survives; one
-// survivor is the answer; otherwise the survivors are re-scored exactly,
-// kappa_j - 2 x.nu_j from the fp64 nu and kappa, ties to the smaller j.
-template <int D, int CP>
-__device__ float approx_score(const uint16_t* __restrict__ hi, const uint16_t* __restrict__ lo,
-                              const double* __restrict__ kap, int j, const float* xv, int lane) {
-  constexpr int kPer = D / 32;
-  const size_t o = static_cast<size_t>(j) * D + kPer * lane;
-  float p = 0.f;
-  if (kPer == 4) {
-    const uint2 h2 = __ldg(reinterpret_cast<const uint2*>(hi + o));
-    const uint2 l2 = __ldg(reinterpret_cast<const uint2*>(lo + o));
-    p = fmaf(xv[0], __uint_as_float(h2.x << 16), p);
-    p = fmaf(xv[0], __uint_as_float(l2.x << 16), p);
-    p = fmaf(xv[1], __uint_as_float(h2.x & 0xffff0000u), p);
-    p = fmaf(xv[1], __uint_as_float(l2.x & 0xffff0000u), p);
-    p = fmaf(xv[2], __uint_as_float(h2.y << 16), p);
-    p = fmaf(xv[2], __uint_as_float(l2.y << 16), p);
-    p = fmaf(xv[3], __uint_as_float(h2.y & 0xffff0000u), p);
-    p = fmaf(xv[3], __uint_as_float(l2.y & 0xffff0000u), p);
-  } else {
-    const uint32_t h1 = __ldg(reinterpret_cast<const uint32_t*>(hi + o));
-    const uint32_t l1 = __ldg(reinterpret_cast<const uint32_t*>(lo + o));
-    p = fmaf(xv[0], __uint_as_float(h1 << 16), p);
-    p = fmaf(xv[0], __uint_as_float(l1 << 16), p);
-    p = fmaf(xv[1], __uint_as_float(h1 & 0xffff0000u), p);
-    p = fmaf(xv[1], __uint_as_float(l1 & 0xffff0000u), p);
-  }
-  for (int s = 16; s > 0; s >>= 1) p += __shfl_xor_sync(0xffffffffu, p, s);
-  return p + static_cast<float>(-0.5 * kap[j]);
-}
-
+// Decides the rows the scorers could not, exactly: score kappa_j - 2 x.nu_j
+// in fp64 over the whole bf16 row (the row is re-read in 16-byte pieces per
+// cluster; they hit L1 and keep the register count low).
 template <int D>
-__device__ __forceinline__ void load_row(const uint16_t* __restrict__ xrow, float* xv, int lane) {
-  xv[0] = xv[1] = xv[2] = xv[3] = 0.f;
-  if (D == 128) {
-    const uint2 w = __ldg(reinterpret_cast<const uint2*>(xrow) + lane);
-    xv[0] = __uint_as_float(w.x << 16);
-    xv[1] = __uint_as_float(w.x & 0xffff0000u);
-    xv[2] = __uint_as_float(w.y << 16);
-    xv[3] = __uint_as_float(w.y & 0xffff0000u);
-  } else {
-    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(xrow) + lane);
-    xv[0] = __uint_as_float(w << 16);
-    xv[1] = __uint_as_float(w & 0xffff0000u);
-  }
-}
-
-// exact score kappa_j - 2 x.nu_j in fp64 (whole warp)
-template <int D>
-__device__ __forceinline__ double exact_score(const double* __restrict__ nu64h, const double* __restrict__ kap,
-                                              int j, const float* xv, int lane) {
-  constexpr int kPer = D / 32;
-  const double* nj = nu64h + static_cast<size_t>(j) * D + kPer * lane;
-  double e = 0.0;
+__device__ __forceinline__ double exact_score(const uint16_t* __restrict__ xrow, const double* __restrict__ nj,
+                                              double kap_j) {
+  double e[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+  for (int i = 0; i < D; i += 8) {
+    const uint4 xw = __ldg(reinterpret_cast<const uint4*>(xrow + i));
+    const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
 #pragma unroll
-  for (int u = 0; u < kPer; ++u) e = fma(static_cast<double>(xv[u]), nj[u], e);
-  for (int s = 16; s > 0; s >>= 1) e += __shfl_xor_sync(0xffffffffu, e, s);
-  return kap[j] - 2.0 * e;
-}
-
-// The label of one row from its listed candidates (n >= 1, ascending): the
-// fp32 scores decide when one candidate stays within E2 of the best,
-// otherwise the survivors are compared exactly (ties to the smaller j).
-template <int D, int CP>
-__device__ int decide_listed(const float* xv, const uint16_t* __restrict__ hi, const uint16_t* __restrict__ lo,
-                             const double* __restrict__ nu64h, const double* __restrict__ kap, float E2,
-                             const int16_t* cand, int n, int lane) {
-  float t[kDeferCand];
-  float T = -INFINITY;
-#pragma unroll
-  for (int q = 0; q < kDeferCand; ++q) {
-    t[q] = q < n ? approx_score<D, CP>(hi, lo, kap, cand[q], xv, lane) : -INFINITY;
-    T = fmaxf(T, t[q]);
-  }
-  int survivors = 0, only = 0;
-#pragma unroll
-  for (int q = 0; q < kDeferCand; ++q)
-    if (q < n && t[q] >= T - E2) {
-      ++survivors;
-      only = cand[q];
-    }
-  if (survivors == 1) return only;
-  double best = INFINITY;
-  int bj = 0;
-#pragma unroll
-  for (int q = 0; q < kDeferCand; ++q) {
-    if (q >= n || t[q] < T - E2) continue;
-    const double sc = exact_score<D>(nu64h, kap, cand[q], xv, lane);
-    if (sc < best) {
-      best = sc;
-      bj = cand[q];
+    for (int u = 0; u < 4; ++u) {
+      const double2 nv = __ldg(reinterpret_cast<const double2*>(nj + i + 2 * u));
+      e[u] = fma(static_cast<double>(__uint_as_float(w[u] << 16)), nv.x, e[u]);
+      e[u] = fma(static_cast<double>(__uint_as_float(w[u] & 0xffff0000u)), nv.y, e[u]);
     }
   }
-  return bj;
+  return kap_j - 2.0 * ((e[0] + e[1]) + (e[2] + e[3]));
 }
 
 // The label of a row against every cluster (rows whose candidates were not
@@ -854,20 +883,7 @@ __device__ int decide_all(const uint16_t* __restrict__ xrow, const double* __res
   double best = INFINITY;
   int bj = 0x7fffffff;
   for (int j = lane; j < C; j += 32) {
-    const double* nj = nu64h + static_cast<size_t>(j) * D;
-    double e[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
-    for (int i = 0; i < D; i += 8) {
-      const uint4 xw = __ldg(reinterpret_cast<const uint4*>(xrow + i));
-      const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const double2 nv = __ldg(reinterpret_cast<const double2*>(nj + i + 2 * u));
-        e[u] = fma(static_cast<double>(__uint_as_float(w[u] << 16)), nv.x, e[u]);
-        e[u] = fma(static_cast<double>(__uint_as_float(w[u] & 0xffff0000u)), nv.y, e[u]);
-      }
-    }
-    const double sc = kap[j] - 2.0 * ((e[0] + e[1]) + (e[2] + e[3]));
+    const double sc = exact_score<D>(xrow, nu64h + static_cast<size_t>(j) * D, kap[j]);
     if (sc < best) {  // j ascends within a lane
       best = sc;
       bj = j;
@@ -884,72 +900,110 @@ __device__ int decide_all(const uint16_t* __restrict__ xrow, const double* __res
   return bj;
 }
 
-// E2 = 2^-16 (|x| max|nu| + max|kappa| / 2) of a row (whole warp)
-__device__ __forceinline__ float row_e2(const float* xv, float max_nrm, float max_kap) {
-  float xx = xv[0] * xv[0] + xv[1] * xv[1] + xv[2] * xv[2] + xv[3] * xv[3];
-  for (int s = 16; s > 0; s >>= 1) xx += __shfl_xor_sync(0xffffffffu, xx, s);
-  return ldexpf(sqrtf(xx) * max_nrm + 0.5f * max_kap, -16);
-}
+// grid: ceil(groups / kFixWarps) blocks of kFixWarps warps, groups = B*H *
+// tiles * 4: one warp per 32-row group. Listed rows: each lane scores one
+// (row, candidate) pair exactly, kappa_j - 2 x.nu_j in fp64, then lane s picks
+// the minimum of row s's pairs (ties to the smaller j). Rows labelled -2 (by
+// the scorers, or here for a list that does not look right): the whole warp
+// compares every cluster (decide_all).
+constexpr int kFixWarps = 8;
+constexpr int kFixItems = kDeferSlots * kDeferCand;  // (row, candidate) pairs of a group, at most
 
-// grid: ceil(BH * ntiles * 4 / 8) blocks of 8 warps, one warp per (head, tile, 32-row group)
 template <int D, int CP>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kFixWarps * 32)
     fixup_kernel(const uint16_t* __restrict__ x, int N, int nv, int C, int BH, int ntiles,
-                 const uint16_t* __restrict__ nu_hi, const uint16_t* __restrict__ nu_lo,
                  const double* __restrict__ nu64, const double* __restrict__ kappa64,
-                 const float* __restrict__ head_max, int32_t* __restrict__ assign,
-                 const int32_t* __restrict__ defer_count, const DeferRec* __restrict__ defer,
-                 int* __restrict__ err) {
-  const int lane = threadIdx.x & 31;
+                 int32_t* __restrict__ assign, const int32_t* __restrict__ defer_count,
+                 const DeferRec* __restrict__ defer, int* __restrict__ err) {
+  __shared__ double sc_s[kFixWarps][kFixItems];
+  __shared__ int j_s[kFixWarps][kFixItems];
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   if (timed_out_before(err)) return;  // the scorers may not have written their lists
-  const long long grp = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  if (grp >= static_cast<long long>(BH) * ntiles * 4) return;
-  const int dc = defer_count[grp];
-  if (dc == 0) return;  // (warp-uniform) nothing was deferred in these 32 rows
-  const int n_def = min(dc & (kDeferAll - 1), kDeferSlots);
-  const int h = static_cast<int>(grp / (static_cast<long long>(ntiles) * 4));
-  const int rem = static_cast<int>(grp - static_cast<long long>(h) * ntiles * 4);
-  const int tt = rem >> 2, lq = rem & 3;
-  const float mn = head_max[2 * h], mk = head_max[2 * h + 1];
-  const uint16_t* hi = nu_hi + static_cast<size_t>(h) * CP * D;
-  const uint16_t* lo = nu_lo + static_cast<size_t>(h) * CP * D;
-  const double* nuh = nu64 + static_cast<size_t>(h) * C * D;
-  const double* kap = kappa64 + static_cast<size_t>(h) * CP;
+  const long long ngrp = static_cast<long long>(BH) * ntiles * 4;
+  const long long g = static_cast<long long>(blockIdx.x) * kFixWarps + wi;
+  if (g >= ngrp) return;  // warp-uniform
+  const int4 dc = *reinterpret_cast<const int4*>(defer_count + g * 4);
+  const int n_def = min(dc.x & (kDeferAll - 1), kDeferSlots);
+  bool any_all = ((dc.x | dc.y | dc.z | dc.w) & kDeferAll) != 0;
+  const int h = static_cast<int>(g / (static_cast<long long>(ntiles) * 4));
+  const int r4 = static_cast<int>(g - static_cast<long long>(h) * ntiles * 4);
+  const int row0 = (r4 >> 2) * kTileRows + (r4 & 3) * 32;  // the group's first token
   int32_t* asg = assign + static_cast<size_t>(h) * nv;
-  const uint16_t* xh = x + static_cast<size_t>(h) * N * D;
-  // listed rows
-  for (int s = 0; s < n_def; ++s) {
-    const DeferRec& rec = defer[grp * kDeferSlots + s];
-    const int tok = rec.tok;
-    if (tok < 0 || tok >= nv) continue;
-    const int n = min(max(rec.n, 1), kDeferCand);
-    int16_t cand[kDeferCand];
-    bool valid = true;  // a list that does not look right falls back to every cluster
+  if (n_def > 0) {
+    const DeferRec* recs = defer + g * kDeferSlots;
+    // lane s < n_def: row s's token and candidate count; a record that does
+    // not look right counts one pair and sends its row to every cluster
+    int tok = -1, n = 0;
+    if (lane < n_def) {
+      tok = recs[lane].tok;
+      n = recs[lane].n;
+      if (tok < row0 || tok >= min(row0 + 32, nv) || n < 2 || n > kDeferCand) n = 0;
+    }
+    int off = n;  // inclusive prefix sum of the counts over the rows
 #pragma unroll
-    for (int q = 0; q < kDeferCand; ++q) {
-      cand[q] = rec.cand[q];
-      valid = valid && (q >= n || (cand[q] >= 0 && cand[q] < C));
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, off, o);
+      if (lane >= o) off += t;
     }
-    int lbl;
-    if (valid) {
-      float xv[4];
-      load_row<D>(xh + static_cast<size_t>(tok) * D, xv, lane);
-      lbl = decide_listed<D, CP>(xv, hi, lo, nuh, kap, row_e2(xv, mn, mk), cand, n, lane);
-    } else {
-      lbl = decide_all<D>(xh + static_cast<size_t>(tok) * D, nuh, kap, C, lane);
+    const int total = __shfl_sync(0xffffffffu, off, 31);
+    off -= n;  // exclusive
+    // every lane runs every round (the shuffles need the whole warp); a lane
+    // past the last pair only shuffles
+    for (int base = 0; base < total; base += 32) {
+      const int it = base + lane;
+      int s = 0;  // the row of pair it: the last s with off_s <= it
+#pragma unroll
+      for (int q = 1; q < kDeferSlots; ++q) {
+        const int off_q = __shfl_sync(0xffffffffu, off, q);
+        if (q < n_def && off_q <= it) s = q;
+      }
+      const int off_s = __shfl_sync(0xffffffffu, off, s);
+      const int t = __shfl_sync(0xffffffffu, tok, s);
+      if (it < total) {
+        const int j = recs[s].cand[it - off_s];
+        double sc = NAN;
+        if (j >= 0 && j < C)
+          sc = exact_score<D>(x + (static_cast<size_t>(h) * N + t) * D,
+                              nu64 + (static_cast<size_t>(h) * C + j) * D, kappa64[static_cast<size_t>(h) * CP + j]);
+        sc_s[wi][it] = sc;
+        j_s[wi][it] = j;
+      }
     }
-    if (lane == 0) asg[tok] = lbl;
+    __syncwarp();
+    if (lane < n_def) {
+      int lbl = -2;  // a bad record or candidate: every cluster
+      if (n > 0) {
+        double best = INFINITY;
+        int bj = 0x7fffffff;
+        bool bad = false;
+        for (int c = 0; c < n; ++c) {
+          const double sc = sc_s[wi][off + c];
+          const int j = j_s[wi][off + c];
+          bad = bad || !(j >= 0 && j < C);
+          if (sc < best || (sc == best && j < bj)) {
+            best = sc;
+            bj = j;
+          }
+        }
+        if (!bad && bj < C) lbl = bj;
+      }
+      if (tok >= row0 && tok < min(row0 + 32, nv)) asg[tok] = lbl;
+      any_all = any_all || lbl == -2;
+    }
+    any_all = __any_sync(0xffffffffu, any_all);
   }
-  // rows whose candidates could not be listed: every cluster
-  if (!(dc & kDeferAll)) return;
-  const int tok = tt * kTileRows + lq * 32 + lane;
+  if (!any_all) return;
+  // rows labelled -2: every cluster, the whole warp per row
+  __syncwarp();
+  const int tok = row0 + lane;
   unsigned all = __ballot_sync(0xffffffffu, tok < nv && asg[tok] == -2);
   while (all) {
     const int l = __ffs(all) - 1;
     all &= all - 1;
-    const int t = tt * kTileRows + lq * 32 + l;
-    const int lbl = decide_all<D>(xh + static_cast<size_t>(t) * D, nuh, kap, C, lane);
-    if (lane == 0) asg[t] = lbl;
+    const int lbl = decide_all<D>(x + (static_cast<size_t>(h) * N + row0 + l) * D,
+                                  nu64 + static_cast<size_t>(h) * C * D, kappa64 + static_cast<size_t>(h) * CP, C,
+                                  lane);
+    if (lane == 0) asg[row0 + l] = lbl;
   }
 }
 
@@ -966,8 +1020,16 @@ constexpr int kUpdTokens = 2048;     // consecutive tokens per CTA
 constexpr int kUpdThreads = 256;
 constexpr int kUpdWarps = kUpdThreads / 32;
 
-__device__ __forceinline__ double flushed(float v) {
-  return fabsf(v) < 5.9604644775390625e-08f ? 0.0 : static_cast<double>(v);  // 2^-24
+// A bf16 value, given as the fp32 bit pattern b (the bf16 in the upper half),
+// to fp64 with |x| < 2^-24 counted as zero, by integer operations: the fp64
+// high word is the sign, the exponent rebased by 1023 - 127 = 896 and the
+// mantissa (a bf16's seven bits fit in it), the low word is zero. (The
+// f32 -> f64 conversion instruction has a fraction of the integer units' rate.)
+__device__ __forceinline__ double bf16_to_f64_flushed(uint32_t b) {
+  const uint32_t mag = b & 0x7fffffffu;
+  uint32_t hi = (b & 0x80000000u) | ((mag >> 3) + (896u << 20));
+  if (mag >= 0x7f800000u) hi = (b & 0x80000000u) | 0x7ff00000u | ((mag & 0x7fffffu) >> 3);  // inf, nan
+  return mag < 0x33800000u ? 0.0 : __hiloint2double(static_cast<int>(hi), 0);  // 0x33800000: 2^-24
 }
 
 __device__ __forceinline__ void red_f64(double* dst, double v) {
@@ -1001,10 +1063,18 @@ __global__ void __launch_bounds__(kUpdThreads)
   const int32_t* a = assign + static_cast<size_t>(h) * nv + c0;
   for (int j = tid; j < C; j += kUpdThreads) cnt[j] = 0;
   __syncthreads();
-  for (int t = tid; t < n; t += kUpdThreads) {
-    const int l = a[t];
-    if (l >= 0 && l < C) atomicAdd(&cnt[l], 1);
-    else report_error(err, kErrBadLabel);
+  // labels come in runs (neighbouring tokens share clusters): lanes with equal
+  // labels add to the shared counters once, through their lowest lane
+  const unsigned lt = (1u << lane) - 1u;
+  for (int t0 = warp * 32; t0 < n; t0 += kUpdThreads) {
+    const int t = t0 + lane;
+    int l = t < n ? a[t] : -1;
+    if (t < n && (l < 0 || l >= C)) {
+      report_error(err, kErrBadLabel);
+      l = -1;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, l);
+    if (l >= 0 && (peers & lt) == 0) atomicAdd(&cnt[l], __popc(peers));
   }
   __syncthreads();
   if (warp == 0) {  // exclusive scan of the counts
@@ -1029,9 +1099,16 @@ __global__ void __launch_bounds__(kUpdThreads)
   __syncthreads();
   for (int j = tid; j < C; j += kUpdThreads) cnt[j] = 0;
   __syncthreads();
-  for (int t = tid; t < n; t += kUpdThreads) {
-    const int l = a[t];
-    if (l >= 0 && l < C) order[base[l] + atomicAdd(&cnt[l], 1)] = static_cast<int16_t>(t);
+  for (int t0 = warp * 32; t0 < n; t0 += kUpdThreads) {
+    const int t = t0 + lane;
+    int l = t < n ? a[t] : -1;
+    if (l >= C) l = -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, l);
+    const int leader = __ffs(peers) - 1;
+    int pos = 0;
+    if (l >= 0 && lane == leader) pos = atomicAdd(&cnt[l], __popc(peers));
+    pos = __shfl_sync(0xffffffffu, pos, leader);
+    if (l >= 0) order[base[l] + pos + __popc(peers & lt)] = static_cast<int16_t>(t);
   }
   __syncthreads();
   const int nvalid = base[C];
@@ -1046,18 +1123,18 @@ __global__ void __launch_bounds__(kUpdThreads)
   }
   int j = lo_j, end = base[j + 1];
   const uint16_t* xc = x + (static_cast<size_t>(h) * N + c0) * D;
-  double acc[kPer];
+  double acc[2][kPer];  // even and odd rows of a batch: two short dependency chains
 #pragma unroll
-  for (int u = 0; u < kPer; ++u) acc[u] = 0.0;
+  for (int u = 0; u < kPer; ++u) acc[0][u] = acc[1][u] = 0.0;
   bool any = false;
   auto flush = [&]() {
     if (any) {
       double* dst = sums + (static_cast<size_t>(h) * C + j) * D + kPer * lane;
 #pragma unroll
-      for (int u = 0; u < kPer; ++u) red_f64(dst + u, acc[u]);
+      for (int u = 0; u < kPer; ++u) red_f64(dst + u, acc[0][u] + acc[1][u]);
     }
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) acc[u] = 0.0;
+    for (int u = 0; u < kPer; ++u) acc[0][u] = acc[1][u] = 0.0;
     any = false;
   };
   for (int pb = p0; pb < p1; pb += kBatch) {
@@ -1086,11 +1163,11 @@ __global__ void __launch_bounds__(kUpdThreads)
         ++j;
         end = base[j + 1];
       }
-      acc[0] += flushed(__uint_as_float(w0[q] << 16));
-      acc[1] += flushed(__uint_as_float(w0[q] & 0xffff0000u));
+      acc[q & 1][0] += bf16_to_f64_flushed(w0[q] << 16);
+      acc[q & 1][1] += bf16_to_f64_flushed(w0[q] & 0xffff0000u);
       if (kPer == 4) {
-        acc[2] += flushed(__uint_as_float(w1[q] << 16));
-        acc[3] += flushed(__uint_as_float(w1[q] & 0xffff0000u));
+        acc[q & 1][2] += bf16_to_f64_flushed(w1[q] << 16);
+        acc[q & 1][3] += bf16_to_f64_flushed(w1[q] & 0xffff0000u);
       }
       any = true;
     }
@@ -1103,18 +1180,84 @@ __global__ void __launch_bounds__(kUpdThreads)
 // grid (C, BH), block d: centroid = fp32(sum / n) (IEEE fp64 division, one
 // rounding), an empty cluster keeps its centroid; clears the sums and the
 // chunk counters for the next half-step.
+// Incremental member sums: the sums and counts of the previous half-step of
+// the same side are kept, and only the tokens whose label changed move: x is
+// added to the new cluster's sum and subtracted from the old one's. Every
+// partial sum is the sum of a set of the same exact fp64 contributions as in
+// update_kernel, so (while N max|x| < 2^22) every addition is exact and the
+// result is bit-identical to summing all members again. prev holds the labels
+// of that half-step and is brought up to date. grid (ceil(nv / 256), B*H),
+// block 256: a warp checks 32 consecutive tokens, then moves each changed
+// row with the whole warp (lane l holds dimensions kPer l .. kPer l + kPer - 1).
+template <int D>
+__global__ void __launch_bounds__(256)
+    update_incr_kernel(const uint16_t* __restrict__ x, int N, int nv, int C,
+                       const int32_t* __restrict__ assign, int32_t* __restrict__ prev,
+                       double* __restrict__ sums, int32_t* __restrict__ counts, int* __restrict__ err) {
+  constexpr int kPer = D / 32;
+  if (timed_out_before(err)) return;  // labels of an aborted step are not to be trusted
+  const int h = blockIdx.y, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t base = static_cast<size_t>(h) * nv;
+  int nw = 0, old = 0;
+  bool moved = false;
+  if (t < nv) {
+    nw = assign[base + t];
+    old = prev[base + t];
+    moved = nw != old;
+    if (moved && (nw < 0 || nw >= C || old < 0 || old >= C)) {
+      report_error(err, kErrBadLabel);
+      moved = false;
+    }
+  }
+  if (moved) {
+    prev[base + t] = nw;
+    atomicAdd(&counts[static_cast<size_t>(h) * C + nw], 1);
+    atomicAdd(&counts[static_cast<size_t>(h) * C + old], -1);
+  }
+  for (unsigned m = __ballot_sync(0xffffffffu, moved); m;) {
+    const int l = __ffs(m) - 1;
+    m &= m - 1;
+    const int tl = t - lane + l;
+    const int to = __shfl_sync(0xffffffffu, nw, l), from = __shfl_sync(0xffffffffu, old, l);
+    const uint16_t* row = x + (static_cast<size_t>(h) * N + tl) * D;
+    double v[kPer];
+    if constexpr (kPer == 4) {
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+      v[0] = bf16_to_f64_flushed(w.x << 16);
+      v[1] = bf16_to_f64_flushed(w.x & 0xffff0000u);
+      v[2] = bf16_to_f64_flushed(w.y << 16);
+      v[3] = bf16_to_f64_flushed(w.y & 0xffff0000u);
+    } else {
+      const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
+      v[0] = bf16_to_f64_flushed(w << 16);
+      v[1] = bf16_to_f64_flushed(w & 0xffff0000u);
+    }
+    double* dst = sums + (static_cast<size_t>(h) * C + to) * D + kPer * lane;
+    double* src = sums + (static_cast<size_t>(h) * C + from) * D + kPer * lane;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      red_f64(dst + u, v[u]);
+      red_f64(src + u, -v[u]);
+    }
+  }
+}
+
+// centroid = fp32(sum / n) where n > 0 (an empty cluster keeps its centroid),
+// sizes = n; resets the chunk counters and, unless `keep` (the call's
+// incremental sums), the sums and counts.
 __global__ void finalize_kernel(double* __restrict__ sums, int32_t* __restrict__ counts,
                                 float* __restrict__ cent, int32_t* __restrict__ sizes,
-                                int32_t* __restrict__ head_next, int C, int d) {
+                                int32_t* __restrict__ head_next, int C, int d, int keep) {
   const int h = blockIdx.y, j = blockIdx.x, i = threadIdx.x;
   const int n = counts[h * C + j];
   const size_t e = (static_cast<size_t>(h) * C + j) * d + i;
   if (n > 0) cent[e] = static_cast<float>(sums[e] / static_cast<double>(n));
-  sums[e] = 0.0;
+  if (!keep) sums[e] = 0.0;
   __syncthreads();
   if (i == 0) {
     sizes[h * C + j] = n;
-    counts[h * C + j] = 0;
+    if (!keep) counts[h * C + j] = 0;
   }
   if (i == 0 && j == 0) head_next[h] = 0;
 }
@@ -1131,10 +1274,11 @@ struct StepWs {
   double* kappa64;
   float* kappa;
   float* nunorm;
+  uint16_t* kimg;
+  float2* numax;
   double* sums;
   int32_t* counts;
   int32_t* head_next;
-  float* head_max;
   float* xnorm;
   int32_t* defer_count;
   DeferRec* defer;
@@ -1156,21 +1300,35 @@ size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out) {
   w.kappa64 = cv.take<double>(static_cast<size_t>(BH) * CP);
   w.kappa = cv.take<float>(static_cast<size_t>(BH) * CP);
   w.nunorm = cv.take<float>(static_cast<size_t>(BH) * CP);
+  w.kimg = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * kExtraK);
+  w.numax = cv.take<float2>(static_cast<size_t>(BH) * (CP / 32));
   w.sums = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
   w.counts = cv.take<int32_t>(static_cast<size_t>(BH) * Cmax);
   w.head_next = cv.take<int32_t>(static_cast<size_t>(BH));
-  w.head_max = cv.take<float>(static_cast<size_t>(BH) * 2);
   w.xnorm = cv.take<float>(static_cast<size_t>(BH) * nv);
-  w.defer_count = cv.take<int32_t>(static_cast<size_t>(BH) * ntiles * 4);
+  w.defer_count = cv.take<int32_t>(static_cast<size_t>(BH) * ntiles * 4 * 4);
   w.defer = cv.take<DeferRec>(static_cast<size_t>(BH) * ntiles * 4 * kDeferSlots);
   if (out) *out = w;
   return cv.used + 256;
 }
 
+// The member sums of one side of a whole svoo_cluster call, kept from one
+// half-step of that side to the next, with the labels they were summed for.
+struct SideSums {
+  double* sums;
+  int32_t* counts;
+  int32_t* prev;
+};
+// kUpdFull: sums from scratch into the step's scratch, cleared afterwards (a
+// lone half-step); kUpdFullKeep: from scratch into the side's kept sums (its
+// first half-step of a call); kUpdIncr: only the changed labels move.
+constexpr int kUpdFull = 0, kUpdFullKeep = 1, kUpdIncr = 2;
+
 template <int D, int CP>
 svoo_status launch_assign(const CUtensorMap& xmap, const svoo_shape* sh, const void* x, int C,
                           const StepWs& w, int32_t* assign, float* xnorm, int xnorm_mode,
-                          int32_t* dev_err, cudaStream_t st) {
+                          double* sums, int32_t* counts, int32_t* prev, int upd, int32_t* dev_err,
+                          cudaStream_t st) {
   const int BH = bh_of(sh), N = sh->N, nv = nvideo_of(sh);
   const size_t smem = 1024 + kAssignHeader + 2 * static_cast<size_t>(kTileRows) * D * 2 +
                       2 * static_cast<size_t>(CP) * D * 2 + (kTileRows + CP) * kExtraK * 2;
@@ -1184,27 +1342,46 @@ svoo_status launch_assign(const CUtensorMap& xmap, const svoo_shape* sh, const v
   const int ntiles = (nv + kTileRows - 1) / kTileRows;
   const long long chunks = static_cast<long long>(BH) * ((ntiles + kChunkTiles - 1) / kChunkTiles);
   const int grid = static_cast<int>(chunks < sms ? chunks : sms);
+  CUtensorMap himap, lomap;
+  if (encode_tiled_2d(&himap, w.nu_hi, static_cast<uint64_t>(BH) * CP, D, CP, 64) != CUDA_SUCCESS ||
+      encode_tiled_2d(&lomap, w.nu_lo, static_cast<uint64_t>(BH) * CP, D, CP, 64) != CUDA_SUCCESS)
+    return SVOO_ERR_CUDA;
   assign_kernel<D, CP><<<grid, kAssignThreads, smem, st>>>(
-      xmap, N, nv, C, BH, w.nu_hi, w.nu_lo, w.kappa64, w.nunorm, w.head_next, assign,
-      w.defer_count, w.defer, xnorm, xnorm_mode, w.head_max, dev_err);
+      xmap, himap, lomap, N, nv, C, BH, w.kimg, w.numax, w.head_next, assign, w.defer_count, w.defer,
+      xnorm, xnorm_mode, dev_err);
   if (cudaGetLastError() != cudaSuccess) return SVOO_ERR_CUDA;
   const long long groups = static_cast<long long>(BH) * ntiles * 4;
-  fixup_kernel<D, CP><<<static_cast<unsigned>((groups + 7) / 8), 256, 0, st>>>(
-      static_cast<const uint16_t*>(x), N, nv, C, BH, ntiles, w.nu_hi, w.nu_lo, w.nu64, w.kappa64,
-      w.head_max, assign, w.defer_count, w.defer, dev_err);
+  fixup_kernel<D, CP><<<static_cast<unsigned>((groups + kFixWarps - 1) / kFixWarps), kFixWarps * 32, 0, st>>>(
+      static_cast<const uint16_t*>(x), N, nv, C, BH, ntiles, w.nu64, w.kappa64, assign, w.defer_count,
+      w.defer, dev_err);
   if (cudaGetLastError() != cudaSuccess) return SVOO_ERR_CUDA;
+  if (upd == kUpdIncr) {
+    update_incr_kernel<D><<<dim3((nv + 255) / 256, BH), 256, 0, st>>>(static_cast<const uint16_t*>(x), N, nv, C,
+                                                                       assign, prev, sums, counts, dev_err);
+    return SVOO_OK;
+  }
   update_kernel<D><<<dim3((nv + kUpdTokens - 1) / kUpdTokens, BH), kUpdThreads, 0, st>>>(
-      static_cast<const uint16_t*>(x), N, nv, C, assign, w.sums, w.counts, dev_err);
+      static_cast<const uint16_t*>(x), N, nv, C, assign, sums, counts, dev_err);
+  if (upd == kUpdFullKeep &&
+      cudaMemcpyAsync(prev, assign, sizeof(int32_t) * BH * static_cast<size_t>(nv), cudaMemcpyDeviceToDevice,
+                      st) != cudaSuccess)
+    return SVOO_ERR_CUDA;
   return SVOO_OK;
 }
 
 // One half-step. metric_cent == nullptr: identity metric. xnorm: per-token
 // |x|^2 store of this side (xnorm_mode kXnormStore / kXnormLoad), else the
-// step computes |x|^2 itself.
+// step computes |x|^2 itself. side (with upd kUpdFullKeep / kUpdIncr): the
+// side's kept sums of a whole call; without it, the step's own scratch.
 svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, int32_t* sizes,
                      int32_t* assign, const float* metric_cent, const int32_t* metric_sizes,
                      int metric_C, const StepWs& w, int32_t* dev_err, cudaStream_t st,
-                     int zero_C, float* xnorm = nullptr, int xnorm_mode = kXnormCompute) {
+                     int zero_C, float* xnorm = nullptr, int xnorm_mode = kXnormCompute,
+                     const SideSums* side = nullptr, int upd = kUpdFull) {
+  double* sums = side ? side->sums : w.sums;
+  int32_t* counts = side ? side->counts : w.counts;
+  int32_t* prev = side ? side->prev : nullptr;
+  if (!side) upd = kUpdFull;
   const int BH = bh_of(sh), d = sh->d, N = sh->N;
   const int CP = score_cols(C);
   // finalize_kernel re-zeroes what a step used, so only the first step of a
@@ -1229,7 +1406,7 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
     return SVOO_ERR_CUDA;
   metric_nu_kernel<<<dim3(CP / 32, BH), 128, metric_nu_smem(d), st>>>(
       metric_cent ? w.M : nullptr, cent, C, CP, d, w.nu64, w.nu_hi, w.nu_lo, w.kappa64, w.kappa,
-      w.nunorm);
+      w.nunorm, w.kimg, w.numax);
   CUtensorMap xmap;
   if (encode_tiled_2d(&xmap, x, static_cast<uint64_t>(BH) * N, d, kTileRows, 64) != CUDA_SUCCESS)
     return SVOO_ERR_CUDA;
@@ -1239,28 +1416,46 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
   }
   svoo_status s;
   if (d == 128)
-    s = CP == 256 ? launch_assign<128, 256>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, dev_err, st)
-                  : launch_assign<128, 128>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, dev_err, st);
+    s = CP == 256 ? launch_assign<128, 256>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, sums, counts, prev, upd,
+                                                   dev_err, st)
+                  : launch_assign<128, 128>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, sums, counts, prev, upd,
+                                                   dev_err, st);
   else
-    s = CP == 256 ? launch_assign<64, 256>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, dev_err, st)
-                  : launch_assign<64, 128>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, dev_err, st);
+    s = CP == 256 ? launch_assign<64, 256>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, sums, counts, prev, upd,
+                                                   dev_err, st)
+                  : launch_assign<64, 128>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, sums, counts, prev, upd,
+                                                   dev_err, st);
   if (s != SVOO_OK) return s;
-  finalize_kernel<<<dim3(C, BH), d, 0, st>>>(w.sums, w.counts, cent, sizes, w.head_next, C, d);
+  finalize_kernel<<<dim3(C, BH), d, 0, st>>>(sums, counts, cent, sizes, w.head_next, C, d,
+                                             upd != kUpdFull ? 1 : 0);
   return launch_status();
 }
 
 bool cluster_counts_ok(int C) { return C >= 1 && C <= 256; }
 
-// Workspace of a whole svoo_cluster call: one half-step's scratch, then the
-// per-token |x|^2 of the queries and of the keys (fp32 [BH][N - n_text] each).
-size_t carve_call(void* ws, const svoo_shape* sh, int Cmax, StepWs* w, float** xn_q, float** xn_k) {
+// Workspace of a whole svoo_cluster call: one half-step's scratch, then per
+// side (queries, keys) the per-token |x|^2 (fp32 [BH][N - n_text]) and the
+// kept member sums (fp64 [BH][C][d]), counts and labels of its last half-step.
+size_t carve_call(void* ws, const svoo_shape* sh, int n_qc, int n_kc, StepWs* w, float** xn_q, float** xn_k,
+                  SideSums* sq, SideSums* sk) {
+  const int Cmax = n_qc > n_kc ? n_qc : n_kc;
   const size_t step = carve_step(ws, bh_of(sh), sh->d, Cmax, nvideo_of(sh), w);
   Carver cv(ws ? static_cast<char*>(ws) + step : nullptr);
-  const size_t n = static_cast<size_t>(bh_of(sh)) * nvideo_of(sh);
+  const size_t BH = static_cast<size_t>(bh_of(sh));
+  const size_t n = BH * nvideo_of(sh);
   float* a = cv.take<float>(n);
   float* b = cv.take<float>(n);
   if (xn_q) *xn_q = a;
   if (xn_k) *xn_k = b;
+  SideSums q, k;
+  q.sums = cv.take<double>(BH * n_qc * sh->d);
+  q.counts = cv.take<int32_t>(BH * n_qc);
+  q.prev = cv.take<int32_t>(n);
+  k.sums = cv.take<double>(BH * n_kc * sh->d);
+  k.counts = cv.take<int32_t>(BH * n_kc);
+  k.prev = cv.take<int32_t>(n);
+  if (sq) *sq = q;
+  if (sk) *sk = k;
   return step + cv.used + 256;
 }
 
@@ -1277,7 +1472,7 @@ using namespace svoo;
 
 extern "C" size_t svoo_cluster_workspace_size(const svoo_shape* shape, int n_qc, int n_kc) {
   if (!shape_ok(shape) || !cluster_counts_ok(n_qc) || !cluster_counts_ok(n_kc)) return 0;
-  return carve_call(nullptr, shape, n_qc > n_kc ? n_qc : n_kc, nullptr, nullptr, nullptr);
+  return carve_call(nullptr, shape, n_qc, n_kc, nullptr, nullptr, nullptr, nullptr, nullptr);
 }
 
 extern "C" svoo_status svoo_cluster_step(const svoo_shape* shape, const void* x, int C, float* cent,
@@ -1313,9 +1508,16 @@ extern "C" svoo_status svoo_cluster(const svoo_shape* shape, const void* q, cons
   const int BH = bh_of(shape), d = shape->d, N = shape->N, nv = nvideo_of(shape);
   StepWs w;
   float *xn_q = nullptr, *xn_k = nullptr;
-  size_t need = carve_call(workspace, shape, n_qc > n_kc ? n_qc : n_kc, &w, &xn_q, &xn_k);
+  SideSums sq, sk;
+  size_t need = carve_call(workspace, shape, n_qc, n_kc, &w, &xn_q, &xn_k, &sq, &sk);
   if (workspace_bytes < need) return SVOO_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // each side's kept sums start empty; its first half-step sums every member
+  if (cudaMemsetAsync(sq.sums, 0, sizeof(double) * BH * static_cast<size_t>(n_qc) * d, st) != cudaSuccess ||
+      cudaMemsetAsync(sq.counts, 0, sizeof(int32_t) * BH * static_cast<size_t>(n_qc), st) != cudaSuccess ||
+      cudaMemsetAsync(sk.sums, 0, sizeof(double) * BH * static_cast<size_t>(n_kc) * d, st) != cudaSuccess ||
+      cudaMemsetAsync(sk.counts, 0, sizeof(int32_t) * BH * static_cast<size_t>(n_kc), st) != cudaSuccess)
+    return SVOO_ERR_CUDA;
   if (!warm) {
     init_centroids_kernel<<<dim3(n_qc, BH), d, 0, st>>>(static_cast<const uint16_t*>(q), N, nv, d, n_qc, q_cent);
     init_centroids_kernel<<<dim3(n_kc, BH), d, 0, st>>>(static_cast<const uint16_t*>(k), N, nv, d, n_kc, k_cent);
@@ -1324,11 +1526,12 @@ extern "C" svoo_status svoo_cluster(const svoo_shape* shape, const void* q, cons
   for (int it = 0; it < iters; ++it) {
     const bool ident = identity || (it == 0 && !warm);
     const int xmode = it == 0 ? kXnormStore : kXnormLoad;  // inputs fixed for the whole call
+    const int upd = it == 0 ? kUpdFullKeep : kUpdIncr;
     svoo_status s = run_step(shape, q, n_qc, q_cent, q_sizes, q_assign, ident ? nullptr : k_cent,
-                             k_sizes, n_kc, w, dev_err, st, it == 0 ? Cmax : 0, xn_q, xmode);
+                             k_sizes, n_kc, w, dev_err, st, it == 0 ? Cmax : 0, xn_q, xmode, &sq, upd);
     if (s != SVOO_OK) return s;
     s = run_step(shape, k, n_kc, k_cent, k_sizes, k_assign, identity ? nullptr : q_cent, q_sizes,
-                 n_qc, w, dev_err, st, 0, xn_k, xmode);
+                 n_qc, w, dev_err, st, 0, xn_k, xmode, &sk, upd);
     if (s != SVOO_OK) return s;
   }
   return SVOO_OK;

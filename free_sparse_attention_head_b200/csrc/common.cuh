@@ -24,9 +24,24 @@ enum : int {
   kErrBadLabel = 1 << 3,        // a cluster label out of range (token skipped)
 };
 
-// About one second at the B200's clock; no legitimate wait inside a CTA's
-// pipeline comes anywhere near it.
+// Budget of a pipeline wait: about one second at the B200's clock; no
+// legitimate wait inside a CTA's pipeline comes anywhere near it. The cleanup
+// waits of an aborting CTA (for TMA copies and MMAs it already issued, which
+// must land before its shared memory and TMEM are released) always get the
+// full second.
+//
+// SVOO_TEST_STALL builds the test-only variant of the library: the pipeline
+// budget shrinks to about 10 ms and each pipelined kernel makes one wait on a
+// barrier that nothing completes, so the timeout path (abort flag, cleanup
+// waits, error bit, fail-fast of the later CTAs) runs for real. The normal
+// build has neither.
+#ifdef SVOO_TEST_STALL
+constexpr long long kWaitBudgetCycles = 20000000LL;
+#else
 constexpr long long kWaitBudgetCycles = 2000000000LL;
+#endif
+constexpr long long kCleanupBudgetCycles = 2000000000LL;
+constexpr uint32_t kSuspendHintNs = 1000000u;  // at most 1 ms, well inside either budget
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -99,17 +114,25 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // Waits for the phase with the given parity to complete. Returns false (and
 // raises *abort) when the budget runs out or another role already aborted;
 // both are checked at least once a millisecond.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          long long budget = kWaitBudgetCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > budget) {
       *abort = 1;
       return false;
     }
   }
+}
+
+// A cleanup wait of an aborting CTA: the full budget, whatever the build, and
+// no abort flag to give up on.
+__device__ __forceinline__ bool mbar_wait_cleanup(uint32_t bar, uint32_t parity) {
+  volatile int never = 0;
+  return mbar_wait(bar, parity, &never, kCleanupBudgetCycles);
 }
 
 // ----------------------------------------------------------------- proxies

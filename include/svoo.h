@@ -143,11 +143,14 @@ size_t svoo_cluster_workspace_size(const svoo_shape *shape, int n_qc, int n_kc);
  * M, nu_j = M mu_j and kappa_j = mu_j . nu_j in
  * fp64. Scores come from tcgen05 MMAs against nu split into two bf16 rows
  * (with kappa folded in); when more than one cluster lies within the MMA's
- * error bound of the best, those candidates are compared again, closer, and
- * in fp64 when still within bound, so the result is that of an fp64
+ * error bound of the best, those candidates (or, when there are many, all
+ * clusters) are compared exactly in fp64, so the result is that of an fp64
  * evaluation. Update: member means from exact sums (see the limits above), so
  * equal labels give bit-identical centroids; an empty cluster keeps its
- * centroid. */
+ * centroid. Each side's first step of a call sums all members; later steps
+ * move only the tokens whose label changed (exact, so the same bits). The
+ * workspace holds those kept sums, so calls sharing one workspace must not
+ * overlap on the GPU. */
 svoo_status svoo_cluster(const svoo_shape *shape, const void *q, const void *k, int n_qc,
                          int n_kc, int iters, int flags, int32_t *q_assign, int32_t *k_assign,
                          float *q_cent, float *k_cent, int32_t *q_sizes, int32_t *k_sizes,

@@ -162,3 +162,11 @@ def test_snr_top_p_rejects_bad_arguments(lib):
         with pytest.raises(svoo.SvooError):
             svoo.snr_top_p(*bad)
     assert lib.svoo_snr_top_p(5, 0, 0.7, 0.9, 1.0, None) == 1
+
+
+def test_stall_library_exports_every_declared_symbol(lib):
+    """The test-only build (SVOO_TEST_STALL) links with the same entry points."""
+    out = os.popen(f"nm -D --defined-only {svoo_build.STALL_LIB}").read()
+    exported = set(re.findall(r"\bT (svoo_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing

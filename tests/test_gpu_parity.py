@@ -204,6 +204,31 @@ def test_cluster_whole(name, metric):
                 assert np.allclose(gc, o[f"{side}_cent"], rtol=1e-4, atol=1e-5)
 
 
+@pytest.mark.parametrize("name", list(SMALL))
+def test_cluster_call_centroids_are_exact_means(name):
+    """A whole call keeps each side's member sums from one half-step to the
+    next and moves only the tokens whose label changed. Being exact, that must
+    give the bits of summing every member again: the returned centroids equal
+    the oracle's update (the exact mean, rounded once) over the call's final
+    labels, and the sizes equal the label counts."""
+    w = SMALL[name]
+    q, k, _ = workload.make_qkv(w)
+    qd, kd, _ = qkv_tensors(q, k, k, w.B, w.H)
+    cl = svoo.cluster(qd, kd, _cfg(w), n_text=w.n_text)
+    torch.cuda.synchronize()
+    svoo.check_device_errors(cl["dev_err"])
+    BH, nv = w.B * w.H, w.n_video
+    for side, x, C in (("q", q, w.n_qc), ("k", k, w.n_kc)):
+        lab = cl[f"{side}_assign"].cpu().numpy().reshape(BH, nv)
+        cent = cl[f"{side}_cent"].cpu().numpy().reshape(BH, C, w.d)
+        sizes = cl[f"{side}_sizes"].cpu().numpy().reshape(BH, C)
+        for h in range(BH):
+            assert np.array_equal(sizes[h], np.bincount(lab[h], minlength=C)), (name, side, h)
+            # empty clusters keep the centroid passed in, so all of them compare
+            want, _ = oracle.update(x[h][:nv], lab[h], cent[h])
+            assert np.array_equal(cent[h].view(np.uint32), want.view(np.uint32)), (name, side, h)
+
+
 def _warm_case(w, cold_rounds=2):
     """The oracle's cold clustering of the call (the previous timestep), and
     the next call's inputs: Q, K drifted by a seeded perturbation."""
