@@ -9,6 +9,8 @@
 //   metric_nu_kernel  nu_j = M mu_j, kappa_j = mu_j . nu_j (fp64), |nu_j|,
 //                     nu_j split into two bf16 rows (hi + lo), -kappa_j/2 in
 //                     three bf16 parts, and per-block maxima for the bound
+//   xnorm_kernel      |x|^2 of every token, once per side and call (the
+//                     assignment's error bound)
 //   assign_kernel     persistent, warp-specialised, dynamically scheduled
 //                     stream of 128-token tiles: tcgen05 MMAs against
 //                     [nu_hi | nu_lo | kappa] into double-buffered TMEM; per
@@ -357,13 +359,16 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 // own head and moves on to the next head with chunks left, so SMs that run
 // this kernel faster take more chunks (on B200 some SMs ran the same tiles up
 // to 1.5x slower than others, so a static split left the fast ones idle).
-// Tile i of a CTA uses X buffer i % 2 and TMEM accumulator i % 2 (CP fp32
-// columns).
+// Tile i of a CTA uses TMEM accumulator i % 2 (CP fp32 columns); its X rows
+// arrive in d/64 stages (128 x 64 bf16, one TMA box each) of a ring of
+// kStages, and a stage goes back to the ring when the MMAs that read it are
+// done (a tcgen05 commit), so copies run two tiles ahead of the MMAs.
 //   scheduler (warp 17) claims the CTA's next chunk while the current one
 //                       runs (one chunk ahead); its lanes probe 32 head
 //                       counters at a time.
-//   producer (warp 0)   streams the chunks' tiles: TMA of the X tile, whose
-//                       head and tile index go into shared memory beside it;
+//   producer (warp 0)   streams the chunks' tiles: TMA of the X stages two
+//                       tiles ahead; per tile, once its accumulator is free,
+//                       publishes the tile's head and index for the scorers;
 //                       on a head change, once the tensor cores are done with
 //                       the old head, TMA of the new head's nu_hi, nu_lo and
 //                       kappa parts; then one tcgen05 chain per tile:
@@ -371,7 +376,8 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 //                       last term a 16-wide K chunk of ones against -kappa_j/2
 //                       split into three bf16 parts, so u_j = x.nu_j - kappa_j/2
 //                       and the score is kappa_j - 2 x.nu_j = -2 u_j.
-//   scorers (warps 1-16) warp w reads TMEM lane quarter w % 4 (32 rows) and
+//   scorers (warps 1-16) never read X (|x|^2 comes from xnorm_kernel); warp w
+//                       reads TMEM lane quarter w % 4 (32 rows) and
 //                       column quarter (w - 1) / 4: each thread loads its row's
 //                       CP/4 scores into registers (then the accumulator goes
 //                       back) and takes the quarter's maximum; the four
@@ -381,11 +387,11 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 //                       contain the exact argmin of the score) and publishes
 //                       their count. From the four counts the four warps take
 //                       the same decision for the row: one candidate is the
-//                       label, written by the warp that holds it; several go
-//                       to the deferred list of the row's 32-row group (up to
-//                       kDeferSlots rows with up to kDeferCand candidates,
-//                       each warp writing its own); the rest (more candidates,
-//                       no free slot, or none at all) get label -2, every
+//                       label, written by the warp that holds it; up to
+//                       kDeferCand (at most kQuarterCand from each quarter)
+//                       are listed for the row in its 32-row group's record,
+//                       each warp writing its own; more, or none at all (only
+//                       with non-finite input), give label -2, every
 //                       cluster. fixup_kernel decides the listed and -2 rows.
 //
 // Error bound: nu_hi + nu_lo equals nu to 2^-18 relative and the three kappa
@@ -394,41 +400,80 @@ inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d
 // |x||nu_j| (1 + 2^-8) + |kappa_j| / 2. E = 2^-13 (|x| max|nu| + max|kappa| / 2)
 // bounds |u_computed - u| with a factor of two to spare.
 
-// |x|^2 of the tokens: computed by the scorers from the X tile (and, with
-// kXnormStore, kept per token for the later half-steps of the same side), or
-// loaded from that store (the inputs do not change between half-steps)
-constexpr int kXnormCompute = 0, kXnormStore = 1, kXnormLoad = 2;
+// |x|^2 of the video tokens of every head (fp32 [BH][nv]), read by the
+// scorers for the error bound. grid (ceil(nv / 32), BH), block 256: a warp
+// takes 4 rows at a time, lane l holding dimensions (D/32) l .. (D/32) l + D/32 - 1.
+template <int D>
+__global__ void __launch_bounds__(256)
+    xnorm_kernel(const uint16_t* __restrict__ x, int N, int nv, float* __restrict__ xnorm) {
+  constexpr int kPer = D / 32;
+  const int h = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r0 = blockIdx.x * 32 + warp * 4;
+  float s[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    s[q] = 0.f;
+    const int r = r0 + q;
+    if (r < nv) {
+      const uint16_t* row = x + (static_cast<size_t>(h) * N + r) * D;
+      if constexpr (kPer == 4) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+        const float a = __uint_as_float(w.x << 16), b = __uint_as_float(w.x & 0xffff0000u);
+        const float c = __uint_as_float(w.y << 16), d = __uint_as_float(w.y & 0xffff0000u);
+        s[q] = fmaf(a, a, b * b) + fmaf(c, c, d * d);
+      } else {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
+        const float a = __uint_as_float(w << 16), b = __uint_as_float(w & 0xffff0000u);
+        s[q] = fmaf(a, a, b * b);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) s[q] += __shfl_xor_sync(0xffffffffu, s[q], o);
+  if (lane < 4 && r0 + lane < nv) {
+    float v = s[0];
+#pragma unroll
+    for (int q = 1; q < 4; ++q)
+      if (lane == q) v = s[q];
+    xnorm[static_cast<size_t>(h) * nv + r0 + lane] = v;
+  }
+}
 
 constexpr int kScorerWarps = 16;
 constexpr int kSchedWarp = 1 + kScorerWarps;
 constexpr int kAssignWarps = 2 + kScorerWarps;
 constexpr int kAssignThreads = kAssignWarps * 32;
 constexpr int kTileRows = 128;
-constexpr int kQuarterCand = 4;      // candidates a quarter may add to a listed row
-constexpr int kDeferSlots = 8;       // listed deferred rows per 32 rows of a tile
-constexpr int kDeferCand = 8;        // candidates of a listed deferred row
+constexpr int kStages = 5;              // X ring: 128-row x 64-column (16 KB) stages
+constexpr int kStageBytes = kTileRows * 64 * 2;
+constexpr int kQuarterCand = 16;     // candidates a quarter may add to a listed row
+constexpr int kDeferCand = 32;       // candidates of a listed row
 constexpr int kDeferAll = 1 << 8;    // defer_count flag: some rows of the group have label -2
 constexpr int kChunkTiles = 4;       // tiles per claimed chunk
-constexpr int kAssignHeader = 6144;  // AssignSmem, keeps the X buffers 1024-aligned
+constexpr int kAssignHeader = 4096;  // AssignSmem, keeps the X stages 1024-aligned
 
-// A row with several candidates, decided by fixup_kernel.
-struct DeferRec {
-  int32_t tok;
-  int32_t n;                   // candidates listed, ascending
-  int16_t cand[kDeferCand];
+// The rows of one 32-row group (a TMEM lane quarter of one tile) that have
+// several candidates, decided by fixup_kernel: row l's count (0: not listed)
+// and its candidates, ascending (cluster ids, < 256).
+struct DeferGroup {
+  uint8_t n[32];
+  uint8_t cand[32][kDeferCand];
 };
 
 struct AssignSmem {
-  uint64_t x_full[2], x_free[2], t_full[2], t_free[2];
+  uint64_t xs_full[kStages], xs_free[kStages];  // X stages: TMA landed / the MMAs reading it are done
+  uint64_t t_full[2], t_free[2];                // TMEM accumulators: MMA done / scores read
+  uint64_t info_full[2];                        // the accumulator's tile (head, index) is published
   uint64_t nu_full, sched_full, sched_free;
 #ifdef SVOO_TEST_STALL
   uint64_t stall;  // test-only: a barrier that nothing completes
 #endif
   uint32_t tmem_base;
   int abort;
-  int tile_h[2], tile_t[2];  // head and tile of each X buffer's tile (head -1: the end)
+  int tile_h[2], tile_t[2];  // head and tile of each accumulator's tile (head -1: the end)
   int sched_h, sched_c;      // the scheduler's claimed chunk (head -1: none left)
-  float xq[4][kTileRows];    // |x|^2 per column quarter's dimensions
   float mq[4][kTileRows];    // per-quarter maxima of u
   uint32_t kc[kTileRows];    // candidates per column quarter, a byte each (saturating)
 };
@@ -471,28 +516,30 @@ __device__ __forceinline__ void mark_ge(uint32_t& m, float v, float thr, uint32_
 }
 
 // grid: min(#SMs, chunks) CTAs, block kAssignThreads. Dynamic smem:
-// [AssignSmem][X 2 x 128 x D bf16][nu_hi CP x D][nu_lo CP x D][ones 128 x 16][kappa parts CP x 16]
+// [AssignSmem][X kStages x 128 x 64 bf16][nu_hi CP x D][nu_lo CP x D][ones 128 x 16][kappa parts CP x 16]
 // kimg: per head the kappa parts tile as it lies in shared memory; numax: per
-// head and 32-cluster block, (max |nu_j|, max |kappa_j|).
+// head and 32-cluster block, (max |nu_j|, max |kappa_j|); xnorm: |x|^2 of the
+// tokens (xnorm_kernel).
 template <int D, int CP>
 __global__ void __launch_bounds__(kAssignThreads, 1)
     assign_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap himap,
                   const __grid_constant__ CUtensorMap lomap, int N, int nv, int C, int BH,
                   const uint16_t* __restrict__ kimg, const float2* __restrict__ numax,
                   int32_t* __restrict__ head_next, int32_t* __restrict__ assign,
-                  int32_t* __restrict__ defer_count, DeferRec* __restrict__ defer,
-                  float* __restrict__ xnorm, int xnorm_mode, int* __restrict__ err) {
+                  int32_t* __restrict__ defer_count, DeferGroup* __restrict__ defer,
+                  const float* __restrict__ xnorm, int* __restrict__ err) {
   constexpr int kQCols = CP / 4;      // score columns per scorer thread
   constexpr int kLoads = kQCols / 32;  // 32-column TMEM loads per thread
-  constexpr uint32_t kXBytes = kTileRows * D * 2;
+  constexpr int kSpt = D / 64;         // X stages per tile
   constexpr uint32_t kNuBytes = CP * D * 2;
   constexpr uint32_t kKBytes = CP * kExtraK * 2;
   static_assert(CP == 128 || CP == 256, "CP must be 128 or 256");
+  static_assert(kSpt >= 1 && 2 * kSpt < kStages, "the ring holds two tiles ahead");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   AssignSmem* S = reinterpret_cast<AssignSmem*>(base);
   uint8_t* xs = base + kAssignHeader;
-  uint8_t* nuh = xs + 2 * kXBytes;
+  uint8_t* nuh = xs + kStages * kStageBytes;
   uint8_t* nul = nuh + kNuBytes;
   uint8_t* ones = nul + kNuBytes;
   uint8_t* kparts = ones + kTileRows * kExtraK * 2;
@@ -505,12 +552,15 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 
   if (tid == 0) {
     S->abort = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&S->xs_full[s]), 1);
+      mbar_init(smem_u32(&S->xs_free[s]), 1);  // a tcgen05.commit
+    }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&S->x_full[b]), 1);
-      // one arrival per warp (after __syncwarp), not per thread
-      mbar_init(smem_u32(&S->x_free[b]), kScorerWarps);
       mbar_init(smem_u32(&S->t_full[b]), 1);
+      // one arrival per warp (after __syncwarp), not per thread
       mbar_init(smem_u32(&S->t_free[b]), kScorerWarps);
+      mbar_init(smem_u32(&S->info_full[b]), 1);
     }
     mbar_init(smem_u32(&S->nu_full), 1);
     mbar_init(smem_u32(&S->sched_full), 1);
@@ -541,11 +591,11 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
   constexpr uint32_t idesc = idesc_bf16_f32(128, CP, false, false);
 
   // producer state (warp 0, lane 0), also read by the abort path below
-  uint32_t tma_pend = 0;         // X buffers with a TMA not yet waited on
-  uint32_t tma_par[2] = {0, 0};  // x_full parity each of them completes
+  uint32_t xs_pend = 0;             // X stages with a TMA not yet waited on
+  uint32_t xs_par[kStages] = {};    // xs_full parity each of them completes
   int mma_last = -1;
-  bool nu_pend = false;          // operand copy not yet waited on
-  uint32_t nu_par = 0;           // nu_full parity of the next operand copy
+  bool nu_pend = false;             // operand copy not yet waited on
+  uint32_t nu_par = 0;              // nu_full parity of the next operand copy
 
   if (warp == kSchedWarp) {
     // ------------------------------------------------------------ scheduler
@@ -587,40 +637,43 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int n_pop = 0, ch = -1, ct = 0, ce = 0;  // current chunk: head, next tile, end
-      // the next tile of the stream: 1 a tile, 0 the end, -1 a timeout
-      auto next_tile = [&](int& h, int& tt) -> int {
-        if (ct >= ce) {
-          if (!mbar_wait(smem_u32(&S->sched_full), n_pop & 1, abort)) return -1;
-          ch = S->sched_h;
-          const int c = S->sched_c;
-          mbar_arrive(smem_u32(&S->sched_free));
-          ++n_pop;
-          if (ch < 0) return 0;
-          ct = c * kChunkTiles;
-          ce = min(ntiles, ct + kChunkTiles);
+      int th[4], tti[4];                       // head and tile of the stream's tiles ii (mod 4)
+      int known = 0;                           // tiles of the stream known so far
+      bool ended = false;
+      // learn tiles up to index want; false on a timeout
+      auto fetch = [&](int want) -> bool {
+        while (!ended && known <= want) {
+          if (ct >= ce) {
+            if (!mbar_wait(smem_u32(&S->sched_full), n_pop & 1, abort)) return false;
+            ch = S->sched_h;
+            const int c = S->sched_c;
+            mbar_arrive(smem_u32(&S->sched_free));
+            ++n_pop;
+            if (ch < 0) {
+              ended = true;
+              break;
+            }
+            ct = c * kChunkTiles;
+            ce = min(ntiles, ct + kChunkTiles);
+          }
+          th[known & 3] = ch;
+          tti[known & 3] = ct++;
+          ++known;
         }
-        h = ch;
-        tt = ct++;
-        return 1;
+        return true;
       };
-      // X tile ii (head -1: the end of the stream, which completes the slot's
-      // x_full without a copy; t_full only ever completes by an MMA commit, so
-      // a wait for a given tile's MMA cannot be completed by this marker)
-      auto issue_tma = [&](int ii, int h, int tt) -> bool {
-        const int b = ii & 1;
-        if (ii >= 2 && !mbar_wait(smem_u32(&S->x_free[b]), ((ii >> 1) - 1) & 1, abort)) return false;
-        S->tile_h[b] = h;
-        S->tile_t[b] = tt;
-        if (h < 0) {
-          mbar_arrive(smem_u32(&S->x_full[b]));
-          return true;
+      // TMA of tile ii's X stages (ring slot of stage q: q % kStages; its
+      // previous occupant, stage q - kStages, is released by an MMA commit)
+      auto load_tile = [&](int ii) -> bool {
+        for (int s = 0; s < kSpt; ++s) {
+          const int q = ii * kSpt + s, slot = q % kStages, use = q / kStages;
+          if (use >= 1 && !mbar_wait(smem_u32(&S->xs_free[slot]), (use - 1) & 1, abort)) return false;
+          mbar_arrive_expect_tx(smem_u32(&S->xs_full[slot]), kStageBytes);
+          tma_load_2d(&xmap, smem_u32(xs + slot * kStageBytes), smem_u32(&S->xs_full[slot]), s * 64,
+                      th[ii & 3] * N + tti[ii & 3] * kTileRows);
+          xs_pend |= 1u << slot;
+          xs_par[slot] = use & 1;
         }
-        mbar_arrive_expect_tx(smem_u32(&S->x_full[b]), kXBytes);
-        for (int s = 0; s < D / 64; ++s)
-          tma_load_2d(&xmap, smem_u32(xs + b * kXBytes + s * kTileRows * 128), smem_u32(&S->x_full[b]),
-                      s * 64, h * N + tt * kTileRows);
-        tma_pend |= 1u << b;
-        tma_par[b] = (ii >> 1) & 1;
         return true;
       };
       // head h's MMA operands, once the tensor cores are done with the old ones
@@ -640,50 +693,64 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         nu_par ^= 1u;
         return true;
       };
+      // publish accumulator ii's tile (head -1: the end of the stream); the
+      // scorers read the slot before they free accumulator ii - 2
+      auto publish = [&](int ii, int h, int tt) -> bool {
+        const int b = ii & 1;
+        if (ii >= 2 && !mbar_wait(smem_u32(&S->t_free[b]), ((ii >> 1) - 1) & 1, abort)) return false;
+        S->tile_h[b] = h;
+        S->tile_t[b] = tt;
+        mbar_arrive(smem_u32(&S->info_full[b]));
+        return true;
+      };
       const uint32_t ha = smem_u32(nuh), la = smem_u32(nul);
       const uint64_t ad_k = plain_desc(smem_u32(ones), 128, 256);
       const uint64_t bd_k = plain_desc(smem_u32(kparts), 128, 256);
-      int hA = -1, tA = 0, loaded_h = -1;
 #ifdef SVOO_TEST_STALL
-      const bool go = mbar_wait(smem_u32(&S->stall), 0, abort);  // nothing completes it
+      bool ok = mbar_wait(smem_u32(&S->stall), 0, abort);  // nothing completes it
 #else
-      constexpr bool go = true;
+      bool ok = true;
 #endif
-      int st = go ? next_tile(hA, tA) : -1;
-      bool ok = st >= 0 && issue_tma(0, st == 1 ? hA : -1, tA);
-      for (int ii = 0; ok && st == 1; ++ii) {
-        int hB = -1, tB = 0;
-        const int st2 = next_tile(hB, tB);
-        if (st2 < 0 || !issue_tma(ii + 1, st2 == 1 ? hB : -1, tB)) break;
-        const int b = ii & 1;
-        if (!mbar_wait(smem_u32(&S->x_full[b]), (ii >> 1) & 1, abort)) break;
-        tma_pend &= ~(1u << b);
-        if (ii >= 2 && !mbar_wait(smem_u32(&S->t_free[b]), ((ii >> 1) - 1) & 1, abort)) break;
-        if (hA != loaded_h) {
-          if (!load_nu(hA)) break;
-          loaded_h = hA;
+      int loaded_h = -1;
+      ok = ok && fetch(1);
+      for (int ii = 0; ok && ii < min(known, 2); ++ii) ok = load_tile(ii);
+      for (int ii = 0; ok; ++ii) {
+        if (ii >= known) {  // the end of the stream
+          publish(ii, -1, 0);
+          break;
+        }
+        const int h = th[ii & 3], tt = tti[ii & 3], b = ii & 1;
+        for (int s = 0; ok && s < kSpt; ++s) {
+          const int q = ii * kSpt + s, slot = q % kStages;
+          ok = mbar_wait(smem_u32(&S->xs_full[slot]), (q / kStages) & 1, abort);
+          if (ok) xs_pend &= ~(1u << slot);
+        }
+        if (!ok || !publish(ii, h, tt)) break;  // also: accumulator b is free again
+        if (h != loaded_h) {
+          if (!load_nu(h)) break;
+          loaded_h = h;
         }
         tc_fence_after();
         const uint32_t dt = tmem + b * CP;
-        const uint32_t xa = smem_u32(xs + b * kXBytes);
+        for (int s = 0; s < kSpt; ++s) {  // stage s: k chunks 4s .. 4s + 3 of the hi and lo products
+          const int slot = (ii * kSpt + s) % kStages;
+          const uint32_t xa = smem_u32(xs + slot * kStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int sub = kk >> 2, off = (kk & 3) * 32;
-          umma_f16(dt, sw128_desc(xa + sub * kTileRows * 128 + off, 16, 1024),
-                   sw128_desc(ha + sub * CP * 128 + off, 16, 1024), idesc, kk > 0);
-        }
+          for (int kq = 0; kq < 4; ++kq)
+            umma_f16(dt, sw128_desc(xa + kq * 32, 16, 1024), sw128_desc(ha + s * CP * 128 + kq * 32, 16, 1024),
+                     idesc, (s > 0 || kq > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int sub = kk >> 2, off = (kk & 3) * 32;
-          umma_f16(dt, sw128_desc(xa + sub * kTileRows * 128 + off, 16, 1024),
-                   sw128_desc(la + sub * CP * 128 + off, 16, 1024), idesc, 1);
+          for (int kq = 0; kq < 4; ++kq)
+            umma_f16(dt, sw128_desc(xa + kq * 32, 16, 1024), sw128_desc(la + s * CP * 128 + kq * 32, 16, 1024),
+                     idesc, 1u);
+          umma_commit(smem_u32(&S->xs_free[slot]));  // the stage goes back once these are done
         }
-        umma_f16(dt, ad_k, bd_k, idesc, 1);
+        umma_f16(dt, ad_k, bd_k, idesc, 1u);
         umma_commit(smem_u32(&S->t_full[b]));
         mma_last = ii;
-        hA = hB;
-        tA = tB;
-        st = st2;
+        // two tiles ahead
+        ok = fetch(ii + 2);
+        if (ok && ii + 2 < known) ok = load_tile(ii + 2);
       }
     }
     __syncwarp();
@@ -694,15 +761,13 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
     const int r = lq * 32 + lane;     // tile row
     const int quad_bar = 1 + lq;      // named barrier of the lane quarter's four warps
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(lq * 32) << 16);
-    const unsigned lanes_below = (1u << lane) - 1u;
     int cur_h = -1;
     float max_nrm = 0.f, max_kap = 0.f;
     for (int ii = 0;; ++ii) {
       const int b = ii & 1;
       const uint32_t ph = (ii >> 1) & 1;
-      // the slot's X copy (or the end-of-stream marker) is there, then, for a
-      // real tile, its MMA is complete
-      bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S->x_full[b]), ph, abort));
+      // the accumulator's tile, then (for a real tile) its MMA is complete
+      bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S->info_full[b]), ph, abort));
       const int h = ok ? S->tile_h[b] : -1;
       const int tt = ok ? S->tile_t[b] : 0;
       if (ok && h >= 0) ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&S->t_full[b]), ph, abort));
@@ -724,30 +789,7 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           max_kap = mk;
           cur_h = h;
         }
-        if (xnorm_mode == kXnormLoad) {
-          // the scorers never read this X tile: it goes back to the producer at once
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&S->x_free[b]));
-          if (tok < nv) xsq = __ldg(xnorm + static_cast<size_t>(h) * nv + tok);
-        } else {  // |x|^2 over this quarter of the dimensions; then the X buffer is free
-          const uint8_t* xb = xs + b * kXBytes;
-          float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-          for (int c = cq * (D / 4); c < (cq + 1) * (D / 4); c += 8) {
-            const uint4 w = *reinterpret_cast<const uint4*>(xb + sw128_offset(r, c, kTileRows));
-            const float f0 = __uint_as_float(w.x << 16), f1 = __uint_as_float(w.x & 0xffff0000u);
-            const float f2 = __uint_as_float(w.y << 16), f3 = __uint_as_float(w.y & 0xffff0000u);
-            const float f4 = __uint_as_float(w.z << 16), f5 = __uint_as_float(w.z & 0xffff0000u);
-            const float f6 = __uint_as_float(w.w << 16), f7 = __uint_as_float(w.w & 0xffff0000u);
-            a0 = fmaf(f0, f0, fmaf(f4, f4, a0));
-            a1 = fmaf(f1, f1, fmaf(f5, f5, a1));
-            a2 = fmaf(f2, f2, fmaf(f6, f6, a2));
-            a3 = fmaf(f3, f3, fmaf(f7, f7, a3));
-          }
-          S->xq[cq][r] = (a0 + a1) + (a2 + a3);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&S->x_free[b]));
-        }
+        if (tok < nv) xsq = __ldg(xnorm + static_cast<size_t>(h) * nv + tok);
         // this quarter's scores into registers; then the accumulator is free
         const uint32_t ta = lane_base + b * CP + cq * kQCols;
         tmem_ld32f(ta, v);
@@ -773,10 +815,6 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       if (named_sync_or(quad_bar, 128, done ? 1 : 0)) break;
       // candidates of this quarter within 2E of the row maximum
       const float U = fmaxf(fmaxf(S->mq[0][r], S->mq[1][r]), fmaxf(S->mq[2][r], S->mq[3][r]));
-      if (xnorm_mode != kXnormLoad) {
-        xsq = (S->xq[0][r] + S->xq[1][r]) + (S->xq[2][r] + S->xq[3][r]);
-        if (xnorm_mode == kXnormStore && cq == 0 && tok < nv) xnorm[static_cast<size_t>(h) * nv + tok] = xsq;
-      }
       const float thr = U - ldexpf(sqrtf(xsq) * max_nrm + 0.5f * max_kap, -12);
       uint32_t mask[kLoads];
 #pragma unroll
@@ -801,9 +839,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
       const int before = cq == 0 ? 0 : cq == 1 ? k0 : cq == 2 ? k0 + k1 : (k0 + k1) + k2;
       const bool row = tok < nv;
       const bool listable = row && total >= 2 && total <= kDeferCand && kmax <= kQuarterCand;
-      const unsigned dm = __ballot_sync(0xffffffffu, listable);
-      const int slot = __popc(dm & lanes_below);
       const long long grp = (static_cast<long long>(h) * ntiles + tt) * 4 + lq;
+      DeferGroup* G = defer + grp;
       int32_t* arow = assign + static_cast<size_t>(h) * nv + tok;
       bool minus2 = false;
       if (row && total == 1) {
@@ -812,36 +849,30 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
           minus2 = j >= C;  // a padding column (only with non-finite input)
           *arow = minus2 ? -2 : j;
         }
-      } else if (listable && slot < kDeferSlots) {
-        DeferRec* dst = defer + grp * kDeferSlots + slot;
-        if (cq == 0) {
-          dst->tok = tok;
-          dst->n = total;
+      } else if (listable) {
+#pragma unroll 1
+        for (int u = 0; u < k; ++u) {
+          const int q = __ffsll(static_cast<long long>(mm)) - 1;
+          mm &= mm - 1;
+          G->cand[lane][before + u] = static_cast<uint8_t>(cq * kQCols + q);
         }
-#pragma unroll
-        for (int u = 0; u < kQuarterCand; ++u) {
-          if (u < k) {
-            const int q = __ffsll(static_cast<long long>(mm)) - 1;
-            mm &= mm - 1;
-            dst->cand[before + u] = static_cast<int16_t>(cq * kQCols + q);
-          }
-        }
-      } else if (row && cq == 0) {  // none, too many, or no free slot: every cluster
+      } else if (row && cq == 0) {  // too many candidates, or none: every cluster
         minus2 = true;
         *arow = -2;
       }
+      if (cq == 0) G->n[lane] = static_cast<uint8_t>(listable ? total : 0);
+      const unsigned dm = __ballot_sync(0xffffffffu, listable);
       const unsigned any2 = __ballot_sync(0xffffffffu, minus2);
       // word cq of the group: the listed rows (word 0) and kDeferAll
-      if (lane == 0)
-        defer_count[grp * 4 + cq] = (cq == 0 ? min(__popc(dm), kDeferSlots) : 0) | (any2 ? kDeferAll : 0);
+      if (lane == 0) defer_count[grp * 4 + cq] = (cq == 0 ? __popc(dm) : 0) | (any2 ? kDeferAll : 0);
     }
   }
   __syncthreads();
   if (*abort && tid == 0) {
     report_error(err, kErrTimeoutCluster);
     // copies and MMAs still in flight complete before the buffers go away
-    for (int b = 0; b < 2; ++b)
-      if (tma_pend & (1u << b)) mbar_wait_cleanup(smem_u32(&S->x_full[b]), tma_par[b]);
+    for (int slot = 0; slot < kStages; ++slot)
+      if (xs_pend & (1u << slot)) mbar_wait_cleanup(smem_u32(&S->xs_full[slot]), xs_par[slot]);
     if (nu_pend) mbar_wait_cleanup(smem_u32(&S->nu_full), nu_par);
     if (mma_last >= 0) mbar_wait_cleanup(smem_u32(&S->t_full[mma_last & 1]), (mma_last >> 1) & 1);
   }
@@ -858,19 +889,29 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 template <int D>
 __device__ __forceinline__ double exact_score(const uint16_t* __restrict__ xrow, const double* __restrict__ nj,
                                               double kap_j) {
-  double e[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
-  for (int i = 0; i < D; i += 8) {
-    const uint4 xw = __ldg(reinterpret_cast<const uint4*>(xrow + i));
-    const uint32_t w[4] = {xw.x, xw.y, xw.z, xw.w};
+  // sixteen independent fp64 FMA chains, summed pairwise: an fp64 FMA's
+  // dependent latency is long on this GPU, so short chains matter more than
+  // the instruction count
+  double e[16];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < 16; ++u) e[u] = 0.0;
+#pragma unroll 2
+  for (int i = 0; i < D; i += 16) {
+    const uint4 xa = __ldg(reinterpret_cast<const uint4*>(xrow + i));
+    const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xrow + i + 8));
+    const uint32_t w[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
       const double2 nv = __ldg(reinterpret_cast<const double2*>(nj + i + 2 * u));
-      e[u] = fma(static_cast<double>(__uint_as_float(w[u] << 16)), nv.x, e[u]);
-      e[u] = fma(static_cast<double>(__uint_as_float(w[u] & 0xffff0000u)), nv.y, e[u]);
+      e[2 * u] = fma(static_cast<double>(__uint_as_float(w[u] << 16)), nv.x, e[2 * u]);
+      e[2 * u + 1] = fma(static_cast<double>(__uint_as_float(w[u] & 0xffff0000u)), nv.y, e[2 * u + 1]);
     }
   }
-  return kap_j - 2.0 * ((e[0] + e[1]) + (e[2] + e[3]));
+#pragma unroll
+  for (int step = 8; step > 0; step >>= 1)
+#pragma unroll
+    for (int u = 0; u < step; ++u) e[u] += e[u + step];
+  return kap_j - 2.0 * e[0];
 }
 
 // The label of a row against every cluster (rows whose candidates were not
@@ -901,44 +942,40 @@ __device__ int decide_all(const uint16_t* __restrict__ xrow, const double* __res
 }
 
 // grid: ceil(groups / kFixWarps) blocks of kFixWarps warps, groups = B*H *
-// tiles * 4: one warp per 32-row group. Listed rows: each lane scores one
-// (row, candidate) pair exactly, kappa_j - 2 x.nu_j in fp64, then lane s picks
-// the minimum of row s's pairs (ties to the smaller j). Rows labelled -2 (by
-// the scorers, or here for a list that does not look right): the whole warp
-// compares every cluster (decide_all).
-constexpr int kFixWarps = 8;
-constexpr int kFixItems = kDeferSlots * kDeferCand;  // (row, candidate) pairs of a group, at most
+// tiles * 4: one warp per 32-row group. Listed rows: the group's (row,
+// candidate) pairs are laid out row after row and each lane scores one pair
+// at a time exactly, kappa_j - 2 x.nu_j in fp64; then lane l picks the minimum
+// of row l's pairs (ties to the smaller j). Rows labelled -2 (by the scorers,
+// or here for a list that does not look right): the whole warp compares every
+// cluster (decide_all).
+constexpr int kFixWarps = 4;
+constexpr int kFixItems = 32 * kDeferCand;  // (row, candidate) pairs of a group, at most
 
 template <int D, int CP>
 __global__ void __launch_bounds__(kFixWarps * 32)
     fixup_kernel(const uint16_t* __restrict__ x, int N, int nv, int C, int BH, int ntiles,
                  const double* __restrict__ nu64, const double* __restrict__ kappa64,
                  int32_t* __restrict__ assign, const int32_t* __restrict__ defer_count,
-                 const DeferRec* __restrict__ defer, int* __restrict__ err) {
+                 const DeferGroup* __restrict__ defer, int* __restrict__ err) {
   __shared__ double sc_s[kFixWarps][kFixItems];
-  __shared__ int j_s[kFixWarps][kFixItems];
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   if (timed_out_before(err)) return;  // the scorers may not have written their lists
   const long long ngrp = static_cast<long long>(BH) * ntiles * 4;
   const long long g = static_cast<long long>(blockIdx.x) * kFixWarps + wi;
   if (g >= ngrp) return;  // warp-uniform
   const int4 dc = *reinterpret_cast<const int4*>(defer_count + g * 4);
-  const int n_def = min(dc.x & (kDeferAll - 1), kDeferSlots);
   bool any_all = ((dc.x | dc.y | dc.z | dc.w) & kDeferAll) != 0;
   const int h = static_cast<int>(g / (static_cast<long long>(ntiles) * 4));
   const int r4 = static_cast<int>(g - static_cast<long long>(h) * ntiles * 4);
   const int row0 = (r4 >> 2) * kTileRows + (r4 & 3) * 32;  // the group's first token
   int32_t* asg = assign + static_cast<size_t>(h) * nv;
-  if (n_def > 0) {
-    const DeferRec* recs = defer + g * kDeferSlots;
-    // lane s < n_def: row s's token and candidate count; a record that does
-    // not look right counts one pair and sends its row to every cluster
-    int tok = -1, n = 0;
-    if (lane < n_def) {
-      tok = recs[lane].tok;
-      n = recs[lane].n;
-      if (tok < row0 || tok >= min(row0 + 32, nv) || n < 2 || n > kDeferCand) n = 0;
-    }
+  const double* nuh = nu64 + static_cast<size_t>(h) * C * D;
+  const double* kap = kappa64 + static_cast<size_t>(h) * CP;
+  if ((dc.x & (kDeferAll - 1)) > 0) {
+    const DeferGroup* G = defer + g;
+    const int tok = row0 + lane;
+    int n = G->n[lane];
+    if (n > kDeferCand || tok >= nv) n = 0;  // not listed (or not a record to trust)
     int off = n;  // inclusive prefix sum of the counts over the rows
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -946,48 +983,42 @@ __global__ void __launch_bounds__(kFixWarps * 32)
       if (lane >= o) off += t;
     }
     const int total = __shfl_sync(0xffffffffu, off, 31);
-    off -= n;  // exclusive
+    off -= n;  // exclusive: row l's pairs are off_l .. off_l + n_l - 1
     // every lane runs every round (the shuffles need the whole warp); a lane
     // past the last pair only shuffles
     for (int base = 0; base < total; base += 32) {
       const int it = base + lane;
-      int s = 0;  // the row of pair it: the last s with off_s <= it
+      int s = 0;  // the row of pair it: the last row l with off_l <= it (rows
+                  // without pairs share the next row's offset, so they are passed over)
 #pragma unroll
-      for (int q = 1; q < kDeferSlots; ++q) {
-        const int off_q = __shfl_sync(0xffffffffu, off, q);
-        if (q < n_def && off_q <= it) s = q;
+      for (int step = 16; step > 0; step >>= 1) {
+        const int off_c = __shfl_sync(0xffffffffu, off, s + step);
+        if (off_c <= it) s += step;
       }
       const int off_s = __shfl_sync(0xffffffffu, off, s);
-      const int t = __shfl_sync(0xffffffffu, tok, s);
       if (it < total) {
-        const int j = recs[s].cand[it - off_s];
-        double sc = NAN;
-        if (j >= 0 && j < C)
-          sc = exact_score<D>(x + (static_cast<size_t>(h) * N + t) * D,
-                              nu64 + (static_cast<size_t>(h) * C + j) * D, kappa64[static_cast<size_t>(h) * CP + j]);
-        sc_s[wi][it] = sc;
-        j_s[wi][it] = j;
+        const int j = G->cand[s][it - off_s];
+        sc_s[wi][it] = j < C ? exact_score<D>(x + (static_cast<size_t>(h) * N + row0 + s) * D,
+                                              nuh + static_cast<size_t>(j) * D, kap[j])
+                             : NAN;
       }
     }
     __syncwarp();
-    if (lane < n_def) {
-      int lbl = -2;  // a bad record or candidate: every cluster
-      if (n > 0) {
-        double best = INFINITY;
-        int bj = 0x7fffffff;
-        bool bad = false;
-        for (int c = 0; c < n; ++c) {
-          const double sc = sc_s[wi][off + c];
-          const int j = j_s[wi][off + c];
-          bad = bad || !(j >= 0 && j < C);
-          if (sc < best || (sc == best && j < bj)) {
-            best = sc;
-            bj = j;
-          }
+    if (n > 0) {
+      double best = INFINITY;
+      int bj = 0x7fffffff;
+      bool bad = false;
+      for (int c = 0; c < n; ++c) {
+        const double sc = sc_s[wi][off + c];
+        const int j = G->cand[lane][c];
+        bad = bad || j >= C;
+        if (sc < best || (sc == best && j < bj)) {
+          best = sc;
+          bj = j;
         }
-        if (!bad && bj < C) lbl = bj;
       }
-      if (tok >= row0 && tok < min(row0 + 32, nv)) asg[tok] = lbl;
+      const int lbl = (!bad && bj < C) ? bj : -2;  // a candidate that does not look right: every cluster
+      asg[tok] = lbl;
       any_all = any_all || lbl == -2;
     }
     any_all = __any_sync(0xffffffffu, any_all);
@@ -1000,9 +1031,7 @@ __global__ void __launch_bounds__(kFixWarps * 32)
   while (all) {
     const int l = __ffs(all) - 1;
     all &= all - 1;
-    const int lbl = decide_all<D>(x + (static_cast<size_t>(h) * N + row0 + l) * D,
-                                  nu64 + static_cast<size_t>(h) * C * D, kappa64 + static_cast<size_t>(h) * CP, C,
-                                  lane);
+    const int lbl = decide_all<D>(x + (static_cast<size_t>(h) * N + row0 + l) * D, nuh, kap, C, lane);
     if (lane == 0) asg[row0 + l] = lbl;
   }
 }
@@ -1021,15 +1050,10 @@ constexpr int kUpdThreads = 256;
 constexpr int kUpdWarps = kUpdThreads / 32;
 
 // A bf16 value, given as the fp32 bit pattern b (the bf16 in the upper half),
-// to fp64 with |x| < 2^-24 counted as zero, by integer operations: the fp64
-// high word is the sign, the exponent rebased by 1023 - 127 = 896 and the
-// mantissa (a bf16's seven bits fit in it), the low word is zero. (The
-// f32 -> f64 conversion instruction has a fraction of the integer units' rate.)
+// to fp64 with |x| < 2^-24 counted as zero.
 __device__ __forceinline__ double bf16_to_f64_flushed(uint32_t b) {
-  const uint32_t mag = b & 0x7fffffffu;
-  uint32_t hi = (b & 0x80000000u) | ((mag >> 3) + (896u << 20));
-  if (mag >= 0x7f800000u) hi = (b & 0x80000000u) | 0x7ff00000u | ((mag & 0x7fffffu) >> 3);  // inf, nan
-  return mag < 0x33800000u ? 0.0 : __hiloint2double(static_cast<int>(hi), 0);  // 0x33800000: 2^-24
+  const float v = __uint_as_float(b);
+  return fabsf(v) < 5.9604644775390625e-08f ? 0.0 : static_cast<double>(v);  // 2^-24
 }
 
 __device__ __forceinline__ void red_f64(double* dst, double v) {
@@ -1040,44 +1064,80 @@ __device__ __forceinline__ void red_s32(int32_t* dst, int v) {
   asm volatile("red.global.add.s32 [%0], %1;" ::"l"(dst), "r"(v) : "memory");
 }
 
-// grid (ceil(nv / kUpdTokens), BH), block kUpdThreads. The CTA groups its
-// kUpdTokens consecutive tokens by label in shared memory (the order inside a
-// cluster is irrelevant: the sums are exact), adds its member counts to
-// counts[h][j], and each warp sums a contiguous run of the grouped order in
-// fp64, adding every cluster's partial sum to sums[h][j]. The rows it reads
-// all lie in the chunk's own contiguous slice of X.
+// grid (ceil(nv / kUpdTokens), BH), block kUpdThreads, one chunk of
+// kUpdTokens consecutive tokens per CTA. prev == nullptr: every token is an
+// entry +x for its label. Otherwise (the incremental update of a whole call:
+// the side's sums and counts of its previous half-step are kept) only the
+// tokens whose label changed since prev are entries, +x for the new label and
+// -x for the old one, and prev is brought up to date; every partial sum is
+// then a sum of the same exact fp64 contributions as a full pass, so the
+// result has the same bits. The CTA groups its entries by cluster in shared
+// memory (the order inside a cluster is irrelevant: the sums are exact), adds
+// each cluster's count change to counts[h][j], and each warp sums a
+// contiguous run of the grouped order in fp64, adding every cluster's
+// partial sum to sums[h][j] once. The rows it reads lie in the chunk's slice
+// of X.
 template <int D>
 __global__ void __launch_bounds__(kUpdThreads)
-    update_kernel(const uint16_t* __restrict__ x, int N, int nv, int C,
-                  const int32_t* __restrict__ assign, double* __restrict__ sums,
-                  int32_t* __restrict__ counts, int* __restrict__ err) {
+    update_kernel(const uint16_t* __restrict__ x, int N, int nv, int C, const int32_t* __restrict__ assign,
+                  int32_t* __restrict__ prev, double* __restrict__ sums, int32_t* __restrict__ counts,
+                  int* __restrict__ err) {
   constexpr int kPer = D / 32;
   constexpr int kBatch = 16;
-  __shared__ int cnt[kMaxClusters];
+  constexpr uint16_t kNeg = 0x8000;  // entry flag: subtract the row
+  __shared__ int cnt[kMaxClusters];   // entries per cluster
+  __shared__ int dlt[kMaxClusters];   // count change per cluster
   __shared__ int base[kMaxClusters + 1];
-  __shared__ int16_t order[kUpdTokens];
+  __shared__ uint16_t order[2 * kUpdTokens];
   const int h = blockIdx.y, c0 = blockIdx.x * kUpdTokens;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (timed_out_before(err)) return;  // labels of an aborted step are not to be trusted
   const int n = min(kUpdTokens, nv - c0);
   const int32_t* a = assign + static_cast<size_t>(h) * nv + c0;
-  for (int j = tid; j < C; j += kUpdThreads) cnt[j] = 0;
+  int32_t* pv = prev ? prev + static_cast<size_t>(h) * nv + c0 : nullptr;
+  for (int j = tid; j < C; j += kUpdThreads) cnt[j] = dlt[j] = 0;
   __syncthreads();
-  // labels come in runs (neighbouring tokens share clusters): lanes with equal
-  // labels add to the shared counters once, through their lowest lane
-  const unsigned lt = (1u << lane) - 1u;
-  for (int t0 = warp * 32; t0 < n; t0 += kUpdThreads) {
-    const int t = t0 + lane;
-    int l = t < n ? a[t] : -1;
+  // a token's entries: (l, +) and, when it moved, (o, -); -1 for none
+  auto entries = [&](int t, int& l, int& o) {
+    l = t < n ? a[t] : -1;
+    o = -1;
     if (t < n && (l < 0 || l >= C)) {
       report_error(err, kErrBadLabel);
       l = -1;
     }
-    const unsigned peers = __match_any_sync(0xffffffffu, l);
-    if (l >= 0 && (peers & lt) == 0) atomicAdd(&cnt[l], __popc(peers));
+    if (pv && t < n) {
+      const int old = pv[t];
+      if (old == l) {
+        l = -1;  // unchanged: no entry
+      } else if (old >= 0 && old < C) {
+        o = old;
+      } else if (l >= 0) {
+        report_error(err, kErrBadLabel);
+        l = -1;
+      }
+    }
+  };
+  // labels come in runs (neighbouring tokens share clusters): lanes with equal
+  // labels add to the shared counters once, through their lowest lane
+  const unsigned lt = (1u << lane) - 1u;
+  for (int t0 = warp * 32; t0 < n; t0 += kUpdThreads) {
+    int l, o;
+    entries(t0 + lane, l, o);
+    const unsigned pl = __match_any_sync(0xffffffffu, l);
+    if (l >= 0 && (pl & lt) == 0) {
+      atomicAdd(&cnt[l], __popc(pl));
+      atomicAdd(&dlt[l], __popc(pl));
+    }
+    if (pv) {
+      const unsigned po = __match_any_sync(0xffffffffu, o);
+      if (o >= 0 && (po & lt) == 0) {
+        atomicAdd(&cnt[o], __popc(po));
+        atomicAdd(&dlt[o], -__popc(po));
+      }
+    }
   }
   __syncthreads();
-  if (warp == 0) {  // exclusive scan of the counts
+  if (warp == 0) {  // exclusive scan of the entry counts
     int run = 0;
     for (int j0 = 0; j0 < C; j0 += 32) {
       const int j = j0 + lane;
@@ -1094,21 +1154,31 @@ __global__ void __launch_bounds__(kUpdThreads)
   }
   __syncthreads();
   for (int j = tid; j < C; j += kUpdThreads) {
-    if (cnt[j] > 0) red_s32(&counts[static_cast<size_t>(h) * C + j], cnt[j]);
+    if (dlt[j] != 0) red_s32(&counts[static_cast<size_t>(h) * C + j], dlt[j]);
+    cnt[j] = 0;
   }
-  __syncthreads();
-  for (int j = tid; j < C; j += kUpdThreads) cnt[j] = 0;
   __syncthreads();
   for (int t0 = warp * 32; t0 < n; t0 += kUpdThreads) {
     const int t = t0 + lane;
-    int l = t < n ? a[t] : -1;
-    if (l >= C) l = -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, l);
-    const int leader = __ffs(peers) - 1;
+    int l, o;
+    entries(t, l, o);
+    const unsigned pl = __match_any_sync(0xffffffffu, l);
+    const int ll = __ffs(pl) - 1;
     int pos = 0;
-    if (l >= 0 && lane == leader) pos = atomicAdd(&cnt[l], __popc(peers));
-    pos = __shfl_sync(0xffffffffu, pos, leader);
-    if (l >= 0) order[base[l] + pos + __popc(peers & lt)] = static_cast<int16_t>(t);
+    if (l >= 0 && lane == ll) pos = atomicAdd(&cnt[l], __popc(pl));
+    pos = __shfl_sync(0xffffffffu, pos, ll);
+    if (l >= 0) order[base[l] + pos + __popc(pl & lt)] = static_cast<uint16_t>(t);
+    if (pv) {
+      const unsigned po = __match_any_sync(0xffffffffu, o);
+      const int lo = __ffs(po) - 1;
+      int pos2 = 0;
+      if (o >= 0 && lane == lo) pos2 = atomicAdd(&cnt[o], __popc(po));
+      pos2 = __shfl_sync(0xffffffffu, pos2, lo);
+      if (o >= 0) {
+        order[base[o] + pos2 + __popc(po & lt)] = static_cast<uint16_t>(t | kNeg);
+        pv[t] = a[t];  // the token's entries are placed: prev catches up
+      }
+    }
   }
   __syncthreads();
   const int nvalid = base[C];
@@ -1123,7 +1193,7 @@ __global__ void __launch_bounds__(kUpdThreads)
   }
   int j = lo_j, end = base[j + 1];
   const uint16_t* xc = x + (static_cast<size_t>(h) * N + c0) * D;
-  double acc[2][kPer];  // even and odd rows of a batch: two short dependency chains
+  double acc[2][kPer];  // even and odd entries of a batch: two short dependency chains
 #pragma unroll
   for (int u = 0; u < kPer; ++u) acc[0][u] = acc[1][u] = 0.0;
   bool any = false;
@@ -1139,12 +1209,15 @@ __global__ void __launch_bounds__(kUpdThreads)
   };
   for (int pb = p0; pb < p1; pb += kBatch) {
     uint32_t w0[kBatch], w1[kBatch];
+    uint32_t neg = 0u;  // bit q: entry q subtracts its row
 #pragma unroll
     for (int q = 0; q < kBatch; ++q) {  // the batch's rows in flight together
       w0[q] = 0u;
       w1[q] = 0u;
       if (pb + q < p1) {
-        const int t = order[pb + q];
+        const uint16_t e = order[pb + q];
+        const int t = e & (kNeg - 1);
+        neg |= (e & kNeg) ? (1u << q) : 0u;
         if (kPer == 4) {
           const uint2 v = __ldg(reinterpret_cast<const uint2*>(xc + static_cast<size_t>(t) * D) + lane);
           w0[q] = v.x;
@@ -1163,84 +1236,18 @@ __global__ void __launch_bounds__(kUpdThreads)
         ++j;
         end = base[j + 1];
       }
-      acc[q & 1][0] += bf16_to_f64_flushed(w0[q] << 16);
-      acc[q & 1][1] += bf16_to_f64_flushed(w0[q] & 0xffff0000u);
+      // +-1 times an exact value is exact
+      const double sg = ((neg >> q) & 1u) ? -1.0 : 1.0;
+      acc[q & 1][0] = fma(sg, bf16_to_f64_flushed(w0[q] << 16), acc[q & 1][0]);
+      acc[q & 1][1] = fma(sg, bf16_to_f64_flushed(w0[q] & 0xffff0000u), acc[q & 1][1]);
       if (kPer == 4) {
-        acc[q & 1][2] += bf16_to_f64_flushed(w1[q] << 16);
-        acc[q & 1][3] += bf16_to_f64_flushed(w1[q] & 0xffff0000u);
+        acc[q & 1][2] = fma(sg, bf16_to_f64_flushed(w1[q] << 16), acc[q & 1][2]);
+        acc[q & 1][3] = fma(sg, bf16_to_f64_flushed(w1[q] & 0xffff0000u), acc[q & 1][3]);
       }
       any = true;
     }
   }
   flush();
-}
-
-// ---------------------------------------------------------------- finalize
-
-// grid (C, BH), block d: centroid = fp32(sum / n) (IEEE fp64 division, one
-// rounding), an empty cluster keeps its centroid; clears the sums and the
-// chunk counters for the next half-step.
-// Incremental member sums: the sums and counts of the previous half-step of
-// the same side are kept, and only the tokens whose label changed move: x is
-// added to the new cluster's sum and subtracted from the old one's. Every
-// partial sum is the sum of a set of the same exact fp64 contributions as in
-// update_kernel, so (while N max|x| < 2^22) every addition is exact and the
-// result is bit-identical to summing all members again. prev holds the labels
-// of that half-step and is brought up to date. grid (ceil(nv / 256), B*H),
-// block 256: a warp checks 32 consecutive tokens, then moves each changed
-// row with the whole warp (lane l holds dimensions kPer l .. kPer l + kPer - 1).
-template <int D>
-__global__ void __launch_bounds__(256)
-    update_incr_kernel(const uint16_t* __restrict__ x, int N, int nv, int C,
-                       const int32_t* __restrict__ assign, int32_t* __restrict__ prev,
-                       double* __restrict__ sums, int32_t* __restrict__ counts, int* __restrict__ err) {
-  constexpr int kPer = D / 32;
-  if (timed_out_before(err)) return;  // labels of an aborted step are not to be trusted
-  const int h = blockIdx.y, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  const size_t base = static_cast<size_t>(h) * nv;
-  int nw = 0, old = 0;
-  bool moved = false;
-  if (t < nv) {
-    nw = assign[base + t];
-    old = prev[base + t];
-    moved = nw != old;
-    if (moved && (nw < 0 || nw >= C || old < 0 || old >= C)) {
-      report_error(err, kErrBadLabel);
-      moved = false;
-    }
-  }
-  if (moved) {
-    prev[base + t] = nw;
-    atomicAdd(&counts[static_cast<size_t>(h) * C + nw], 1);
-    atomicAdd(&counts[static_cast<size_t>(h) * C + old], -1);
-  }
-  for (unsigned m = __ballot_sync(0xffffffffu, moved); m;) {
-    const int l = __ffs(m) - 1;
-    m &= m - 1;
-    const int tl = t - lane + l;
-    const int to = __shfl_sync(0xffffffffu, nw, l), from = __shfl_sync(0xffffffffu, old, l);
-    const uint16_t* row = x + (static_cast<size_t>(h) * N + tl) * D;
-    double v[kPer];
-    if constexpr (kPer == 4) {
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(row) + lane);
-      v[0] = bf16_to_f64_flushed(w.x << 16);
-      v[1] = bf16_to_f64_flushed(w.x & 0xffff0000u);
-      v[2] = bf16_to_f64_flushed(w.y << 16);
-      v[3] = bf16_to_f64_flushed(w.y & 0xffff0000u);
-    } else {
-      const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
-      v[0] = bf16_to_f64_flushed(w << 16);
-      v[1] = bf16_to_f64_flushed(w & 0xffff0000u);
-    }
-    double* dst = sums + (static_cast<size_t>(h) * C + to) * D + kPer * lane;
-    double* src = sums + (static_cast<size_t>(h) * C + from) * D + kPer * lane;
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      red_f64(dst + u, v[u]);
-      red_f64(src + u, -v[u]);
-    }
-  }
 }
 
 // centroid = fp32(sum / n) where n > 0 (an empty cluster keeps its centroid),
@@ -1281,7 +1288,7 @@ struct StepWs {
   int32_t* head_next;
   float* xnorm;
   int32_t* defer_count;
-  DeferRec* defer;
+  DeferGroup* defer;
 };
 
 // columns of the scoring MMA: the cluster count padded so that four threads
@@ -1307,7 +1314,7 @@ size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out) {
   w.head_next = cv.take<int32_t>(static_cast<size_t>(BH));
   w.xnorm = cv.take<float>(static_cast<size_t>(BH) * nv);
   w.defer_count = cv.take<int32_t>(static_cast<size_t>(BH) * ntiles * 4 * 4);
-  w.defer = cv.take<DeferRec>(static_cast<size_t>(BH) * ntiles * 4 * kDeferSlots);
+  w.defer = cv.take<DeferGroup>(static_cast<size_t>(BH) * ntiles * 4);
   if (out) *out = w;
   return cv.used + 256;
 }
@@ -1326,11 +1333,10 @@ constexpr int kUpdFull = 0, kUpdFullKeep = 1, kUpdIncr = 2;
 
 template <int D, int CP>
 svoo_status launch_assign(const CUtensorMap& xmap, const svoo_shape* sh, const void* x, int C,
-                          const StepWs& w, int32_t* assign, float* xnorm, int xnorm_mode,
-                          double* sums, int32_t* counts, int32_t* prev, int upd, int32_t* dev_err,
-                          cudaStream_t st) {
+                          const StepWs& w, int32_t* assign, const float* xnorm, double* sums,
+                          int32_t* counts, int32_t* prev, int upd, int32_t* dev_err, cudaStream_t st) {
   const int BH = bh_of(sh), N = sh->N, nv = nvideo_of(sh);
-  const size_t smem = 1024 + kAssignHeader + 2 * static_cast<size_t>(kTileRows) * D * 2 +
+  const size_t smem = 1024 + kAssignHeader + static_cast<size_t>(kStages) * kStageBytes +
                       2 * static_cast<size_t>(CP) * D * 2 + (kTileRows + CP) * kExtraK * 2;
   if (cudaFuncSetAttribute(assign_kernel<D, CP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
@@ -1348,20 +1354,16 @@ svoo_status launch_assign(const CUtensorMap& xmap, const svoo_shape* sh, const v
     return SVOO_ERR_CUDA;
   assign_kernel<D, CP><<<grid, kAssignThreads, smem, st>>>(
       xmap, himap, lomap, N, nv, C, BH, w.kimg, w.numax, w.head_next, assign, w.defer_count, w.defer,
-      xnorm, xnorm_mode, dev_err);
+      xnorm, dev_err);
   if (cudaGetLastError() != cudaSuccess) return SVOO_ERR_CUDA;
   const long long groups = static_cast<long long>(BH) * ntiles * 4;
   fixup_kernel<D, CP><<<static_cast<unsigned>((groups + kFixWarps - 1) / kFixWarps), kFixWarps * 32, 0, st>>>(
       static_cast<const uint16_t*>(x), N, nv, C, BH, ntiles, w.nu64, w.kappa64, assign, w.defer_count,
       w.defer, dev_err);
   if (cudaGetLastError() != cudaSuccess) return SVOO_ERR_CUDA;
-  if (upd == kUpdIncr) {
-    update_incr_kernel<D><<<dim3((nv + 255) / 256, BH), 256, 0, st>>>(static_cast<const uint16_t*>(x), N, nv, C,
-                                                                       assign, prev, sums, counts, dev_err);
-    return SVOO_OK;
-  }
   update_kernel<D><<<dim3((nv + kUpdTokens - 1) / kUpdTokens, BH), kUpdThreads, 0, st>>>(
-      static_cast<const uint16_t*>(x), N, nv, C, assign, sums, counts, dev_err);
+      static_cast<const uint16_t*>(x), N, nv, C, assign, upd == kUpdIncr ? prev : nullptr, sums, counts,
+      dev_err);
   if (upd == kUpdFullKeep &&
       cudaMemcpyAsync(prev, assign, sizeof(int32_t) * BH * static_cast<size_t>(nv), cudaMemcpyDeviceToDevice,
                       st) != cudaSuccess)
@@ -1369,15 +1371,27 @@ svoo_status launch_assign(const CUtensorMap& xmap, const svoo_shape* sh, const v
   return SVOO_OK;
 }
 
-// One half-step. metric_cent == nullptr: identity metric. xnorm: per-token
-// |x|^2 store of this side (xnorm_mode kXnormStore / kXnormLoad), else the
-// step computes |x|^2 itself. side (with upd kUpdFullKeep / kUpdIncr): the
-// side's kept sums of a whole call; without it, the step's own scratch.
+// |x|^2 of the video tokens of x into xn (fp32 [BH][nv]).
+svoo_status launch_xnorm(const svoo_shape* sh, const void* x, float* xn, cudaStream_t st) {
+  const int BH = bh_of(sh), nv = nvideo_of(sh);
+  const dim3 grid((nv + 31) / 32, BH);
+  if (sh->d == 128)
+    xnorm_kernel<128><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), sh->N, nv, xn);
+  else
+    xnorm_kernel<64><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(x), sh->N, nv, xn);
+  return cudaGetLastError() == cudaSuccess ? SVOO_OK : SVOO_ERR_CUDA;
+}
+
+// One half-step. metric_cent == nullptr: identity metric. xnorm: |x|^2 of
+// this side's tokens, already computed for the whole call; without it the
+// step computes it into its own scratch. side (with upd kUpdFullKeep /
+// kUpdIncr): the side's kept sums of a whole call; without it, the step's own
+// scratch.
 svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, int32_t* sizes,
                      int32_t* assign, const float* metric_cent, const int32_t* metric_sizes,
                      int metric_C, const StepWs& w, int32_t* dev_err, cudaStream_t st,
-                     int zero_C, float* xnorm = nullptr, int xnorm_mode = kXnormCompute,
-                     const SideSums* side = nullptr, int upd = kUpdFull) {
+                     int zero_C, const float* xnorm = nullptr, const SideSums* side = nullptr,
+                     int upd = kUpdFull) {
   double* sums = side ? side->sums : w.sums;
   int32_t* counts = side ? side->counts : w.counts;
   int32_t* prev = side ? side->prev : nullptr;
@@ -1410,21 +1424,17 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
   CUtensorMap xmap;
   if (encode_tiled_2d(&xmap, x, static_cast<uint64_t>(BH) * N, d, kTileRows, 64) != CUDA_SUCCESS)
     return SVOO_ERR_CUDA;
-  if (!xnorm) {  // a lone half-step computes |x|^2 from the tiles
+  if (!xnorm) {  // a lone half-step
+    if (launch_xnorm(sh, x, w.xnorm, st) != SVOO_OK) return SVOO_ERR_CUDA;
     xnorm = w.xnorm;
-    xnorm_mode = kXnormCompute;
   }
   svoo_status s;
   if (d == 128)
-    s = CP == 256 ? launch_assign<128, 256>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, sums, counts, prev, upd,
-                                                   dev_err, st)
-                  : launch_assign<128, 128>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, sums, counts, prev, upd,
-                                                   dev_err, st);
+    s = CP == 256 ? launch_assign<128, 256>(xmap, sh, x, C, w, assign, xnorm, sums, counts, prev, upd, dev_err, st)
+                  : launch_assign<128, 128>(xmap, sh, x, C, w, assign, xnorm, sums, counts, prev, upd, dev_err, st);
   else
-    s = CP == 256 ? launch_assign<64, 256>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, sums, counts, prev, upd,
-                                                   dev_err, st)
-                  : launch_assign<64, 128>(xmap, sh, x, C, w, assign, xnorm, xnorm_mode, sums, counts, prev, upd,
-                                                   dev_err, st);
+    s = CP == 256 ? launch_assign<64, 256>(xmap, sh, x, C, w, assign, xnorm, sums, counts, prev, upd, dev_err, st)
+                  : launch_assign<64, 128>(xmap, sh, x, C, w, assign, xnorm, sums, counts, prev, upd, dev_err, st);
   if (s != SVOO_OK) return s;
   finalize_kernel<<<dim3(C, BH), d, 0, st>>>(sums, counts, cent, sizes, w.head_next, C, d,
                                              upd != kUpdFull ? 1 : 0);
@@ -1523,15 +1533,17 @@ extern "C" svoo_status svoo_cluster(const svoo_shape* shape, const void* q, cons
     init_centroids_kernel<<<dim3(n_kc, BH), d, 0, st>>>(static_cast<const uint16_t*>(k), N, nv, d, n_kc, k_cent);
   }
   const int Cmax = n_qc > n_kc ? n_qc : n_kc;
+  // |x|^2 of both sides' tokens (the inputs do not change during the call)
+  if (launch_xnorm(shape, q, xn_q, st) != SVOO_OK || launch_xnorm(shape, k, xn_k, st) != SVOO_OK)
+    return SVOO_ERR_CUDA;
   for (int it = 0; it < iters; ++it) {
     const bool ident = identity || (it == 0 && !warm);
-    const int xmode = it == 0 ? kXnormStore : kXnormLoad;  // inputs fixed for the whole call
     const int upd = it == 0 ? kUpdFullKeep : kUpdIncr;
     svoo_status s = run_step(shape, q, n_qc, q_cent, q_sizes, q_assign, ident ? nullptr : k_cent,
-                             k_sizes, n_kc, w, dev_err, st, it == 0 ? Cmax : 0, xn_q, xmode, &sq, upd);
+                             k_sizes, n_kc, w, dev_err, st, it == 0 ? Cmax : 0, xn_q, &sq, upd);
     if (s != SVOO_OK) return s;
     s = run_step(shape, k, n_kc, k_cent, k_sizes, k_assign, identity ? nullptr : q_cent, q_sizes,
-                 n_qc, w, dev_err, st, 0, xn_k, xmode, &sk, upd);
+                 n_qc, w, dev_err, st, 0, xn_k, &sk, upd);
     if (s != SVOO_OK) return s;
   }
   return SVOO_OK;
