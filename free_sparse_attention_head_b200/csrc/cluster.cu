@@ -240,9 +240,27 @@ __global__ void __launch_bounds__(128)
     cp_async_commit();
   };
   if (Mh) stage(0);
-  for (int e = threadIdx.x; e < 32 * d; e += blockDim.x) {
-    const int r = e / d, c = e % d;
-    mu[r * kNuMuStride + c] = (j0 + r < C) ? static_cast<double>(cent[(static_cast<size_t>(h) * C + j0 + r) * d + c]) : 0.0;
+  {  // the block's 32 centroids, all float4 loads in flight before any store
+    constexpr int kLd = 32 * 128 / 4 / 128;  // float4 per thread (d = 128; half of them for d = 64)
+    float4 f[kLd];
+#pragma unroll
+    for (int q = 0; q < kLd; ++q) {
+      const int e = (threadIdx.x + q * 128) * 4, r = e / d, c = e % d;
+      f[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < 32 * d && j0 + r < C)
+        f[q] = __ldg(reinterpret_cast<const float4*>(cent + (static_cast<size_t>(h) * C + j0 + r) * d + c));
+    }
+#pragma unroll
+    for (int q = 0; q < kLd; ++q) {
+      const int e = (threadIdx.x + q * 128) * 4, r = e / d, c = e % d;
+      if (e < 32 * d) {
+        double* m = mu + r * kNuMuStride + c;
+        m[0] = f[q].x;
+        m[1] = f[q].y;
+        m[2] = f[q].z;
+        m[3] = f[q].w;
+      }
+    }
   }
   const int nd = d == 128 ? 4 : 2;  // dimensions per lane
   const int dim[4] = {2 * lane, 2 * lane + 1, 64 + 2 * lane, 65 + 2 * lane};
@@ -943,21 +961,24 @@ __device__ int decide_all(const uint16_t* __restrict__ xrow, const double* __res
 
 // grid: ceil(groups / kFixWarps) blocks of kFixWarps warps, groups = B*H *
 // tiles * 4: one warp per 32-row group. Listed rows: the group's (row,
-// candidate) pairs are laid out row after row and each lane scores one pair
-// at a time exactly, kappa_j - 2 x.nu_j in fp64; then lane l picks the minimum
-// of row l's pairs (ties to the smaller j). Rows labelled -2 (by the scorers,
-// or here for a list that does not look right): the whole warp compares every
-// cluster (decide_all).
+// candidate) pairs are laid out row after row, 32 per round, and each lane
+// scores one pair exactly, kappa_j - 2 x.nu_j in fp64; a segmented minimum
+// over the lanes of each row's run (ties to the smaller j) goes to the row's
+// own lane, which keeps the row's best over the rounds. Rows labelled -2 (by
+// the scorers, or here for a list that does not look right): the whole warp
+// compares every cluster (decide_all).
 constexpr int kFixWarps = 4;
-constexpr int kFixItems = 32 * kDeferCand;  // (row, candidate) pairs of a group, at most
+
+__device__ __forceinline__ bool better(double sa, int ja, double sb, int jb) {
+  return sa < sb || (sa == sb && ja < jb);  // NaN never wins
+}
 
 template <int D, int CP>
-__global__ void __launch_bounds__(kFixWarps * 32)
+__global__ void __launch_bounds__(kFixWarps * 32, 5)
     fixup_kernel(const uint16_t* __restrict__ x, int N, int nv, int C, int BH, int ntiles,
                  const double* __restrict__ nu64, const double* __restrict__ kappa64,
                  int32_t* __restrict__ assign, const int32_t* __restrict__ defer_count,
                  const DeferGroup* __restrict__ defer, int* __restrict__ err) {
-  __shared__ double sc_s[kFixWarps][kFixItems];
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   if (timed_out_before(err)) return;  // the scorers may not have written their lists
   const long long ngrp = static_cast<long long>(BH) * ntiles * 4;
@@ -984,8 +1005,10 @@ __global__ void __launch_bounds__(kFixWarps * 32)
     }
     const int total = __shfl_sync(0xffffffffu, off, 31);
     off -= n;  // exclusive: row l's pairs are off_l .. off_l + n_l - 1
-    // every lane runs every round (the shuffles need the whole warp); a lane
-    // past the last pair only shuffles
+    double best = INFINITY;  // this lane's row, over the rounds
+    int bj = 0x7fffffff;
+    bool bad = false;
+    // every lane runs every round (the shuffles need the whole warp)
     for (int base = 0; base < total; base += 32) {
       const int it = base + lane;
       int s = 0;  // the row of pair it: the last row l with off_l <= it (rows
@@ -996,27 +1019,45 @@ __global__ void __launch_bounds__(kFixWarps * 32)
         if (off_c <= it) s += step;
       }
       const int off_s = __shfl_sync(0xffffffffu, off, s);
+      double sc = NAN;
+      int j = 0x7fffffff;
       if (it < total) {
-        const int j = G->cand[s][it - off_s];
-        sc_s[wi][it] = j < C ? exact_score<D>(x + (static_cast<size_t>(h) * N + row0 + s) * D,
-                                              nuh + static_cast<size_t>(j) * D, kap[j])
-                             : NAN;
+        j = G->cand[s][it - off_s];
+        if (j < C)
+          sc = exact_score<D>(x + (static_cast<size_t>(h) * N + row0 + s) * D, nuh + static_cast<size_t>(j) * D,
+                              kap[j]);
+        else
+          j = -1;  // a candidate that does not look right
       }
-    }
-    __syncwarp();
-    if (n > 0) {
-      double best = INFINITY;
-      int bj = 0x7fffffff;
-      bool bad = false;
-      for (int c = 0; c < n; ++c) {
-        const double sc = sc_s[wi][off + c];
-        const int j = G->cand[lane][c];
-        bad = bad || j >= C;
-        if (sc < best || (sc == best && j < bj)) {
-          best = sc;
-          bj = j;
+      // segmented minimum: a row's pairs are a run of consecutive lanes
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double sc2 = __shfl_down_sync(0xffffffffu, sc, o);
+        const int j2 = __shfl_down_sync(0xffffffffu, j, o);
+        const int s2 = __shfl_down_sync(0xffffffffu, s, o);
+        const int it2 = it + o;
+        if (lane + o < 32 && it2 < total && s2 == s) {
+          if (j2 < 0 || j < 0) j = -1;  // a bad candidate anywhere in the row's run
+          else if (better(sc2, j2, sc, j)) {
+            sc = sc2;
+            j = j2;
+          }
         }
       }
+      // the run of row `lane` in this round starts at lane max(off - base, 0)
+      const bool mine = n > 0 && off < base + 32 && off + n > base;
+      const int head = max(off - base, 0);
+      const double rs = __shfl_sync(0xffffffffu, sc, mine ? head : lane);
+      const int rj = __shfl_sync(0xffffffffu, j, mine ? head : lane);
+      if (mine) {
+        if (rj < 0) bad = true;
+        else if (better(rs, rj, best, bj)) {
+          best = rs;
+          bj = rj;
+        }
+      }
+    }
+    if (n > 0) {
       const int lbl = (!bad && bj < C) ? bj : -2;  // a candidate that does not look right: every cluster
       asg[tok] = lbl;
       any_all = any_all || lbl == -2;
