@@ -43,24 +43,29 @@ __global__ void init_centroids_kernel(const uint16_t* __restrict__ x, int N, int
 
 // ---------------------------------------------------------------- metric
 
-// M[h] = sum_b n_b c_b c_b^T / sum_b n_b in fp64. grid (T*(T+1)/2, BH) with
-// T = d/64 output blocks of 64 x 64 per side (upper triangle only; an
-// off-diagonal block is written to both (i, j) and (j, i), so M is exactly
-// symmetric), block 512 = two groups of 16 x 16 threads that take alternate
-// 32-cluster chunks (their partial blocks are added at the end, group 0's
-// plus group 1's); thread (ty, tx) of a group owns rows i0 + 4ty .. +3 and
-// columns j0 + {2tx, 2tx+1, 32+2tx, 33+2tx}. The next chunk's values are
-// fetched into registers while the current one is used.
+// M[h] = sum_b n_b c_b c_b^T / sum_b n_b in fp64. grid (T*(T+1)/2, BH,
+// kMSplit) with T = d/64 output blocks of 64 x 64 per side (upper triangle
+// only; an off-diagonal block is written to both (i, j) and (j, i), so M is
+// exactly symmetric); slice z of the grid sums the z-th quarter of the
+// clusters. Block 512 = two groups of 16 x 16 threads that take alternate
+// 32-cluster chunks of the slice; thread (ty, tx) of a group owns rows
+// i0 + 4ty .. +3 and columns j0 + {2tx, 2tx+1, 32+2tx, 33+2tx}. Each slice
+// writes its partial block (group 0's plus group 1's); the slice that
+// finishes last adds the kMSplit partials in slice order, so the result does
+// not depend on which slice ran when. The next chunk's values are fetched
+// into registers while the current one is used.
 constexpr int kMBlk = 64;
 constexpr int kMChunk = 32;
 constexpr int kMThreads = 512;
+constexpr int kMSplit = 4;
 
 __global__ void __launch_bounds__(kMThreads)
     metric_m_kernel(const float* __restrict__ cent, const int32_t* __restrict__ sizes, int C, int d,
-                    double* __restrict__ M) {
+                    double* __restrict__ M, double* __restrict__ mpart, int32_t* __restrict__ mticket) {
   extern __shared__ __align__(16) double msm[];   // per group: as[32][64], bs[32][64]
   __shared__ long long total_s;
-  const int h = blockIdx.y, T = d / kMBlk;
+  __shared__ int last_s;
+  const int h = blockIdx.y, T = d / kMBlk, z = blockIdx.z;
   int t = blockIdx.x, bi = 0;
   while (t >= T - bi) {  // upper-triangle block index -> (bi, bj), bi <= bj
     t -= T - bi;
@@ -98,11 +103,26 @@ __global__ void __launch_bounds__(kMThreads)
   for (int u = 0; u < 4; ++u)
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc[u][v] = 0.0;
+  // this slice's chunks: kc0 .. kc1 - 1
   const int nchunks = (C + kMChunk - 1) / kMChunk;
-  const int rounds = (nchunks + 1) / 2;  // both groups run the same number of rounds
-  fetch(grp * kMChunk);
+  const int per = (nchunks + static_cast<int>(gridDim.z) - 1) / static_cast<int>(gridDim.z);
+  const int kc0 = min(nchunks, z * per), kc1 = min(nchunks, kc0 + per);
+  const int cend = min(C, kc1 * kMChunk);  // the slice's clusters end here
+  const int rounds = (kc1 - kc0 + 1) / 2;  // both groups run the same number of rounds
+  auto fetch_in = [&](int b0) {
+    if (b0 < cend) {
+      fetch(b0);
+    } else {
+#pragma unroll
+      for (int q = 0; q < kPer; ++q) {
+        fa[q] = fb[q] = 0.f;
+        nb_[q] = 0;
+      }
+    }
+  };
+  fetch_in((kc0 + grp) * kMChunk);
   for (int rd = 0; rd < rounds; ++rd) {
-    const int b0 = (2 * rd + grp) * kMChunk;
+    const int b0 = (kc0 + 2 * rd + grp) * kMChunk;
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
@@ -111,8 +131,8 @@ __global__ void __launch_bounds__(kMThreads)
       bs[e] = static_cast<double>(fb[q]);
     }
     __syncthreads();
-    if (b0 + 2 * kMChunk < C) fetch(b0 + 2 * kMChunk);
-    const int nb = max(0, min(kMChunk, C - b0));
+    fetch_in(b0 + 2 * kMChunk);
+    const int nb = max(0, min(kMChunk, cend - b0));
     for (int bb = 0; bb < nb; ++bb) {
       const double2 a01 = *reinterpret_cast<const double2*>(&as[bb * kMBlk + 4 * ty]);
       const double2 a23 = *reinterpret_cast<const double2*>(&as[bb * kMBlk + 4 * ty + 2]);
@@ -142,16 +162,48 @@ __global__ void __launch_bounds__(kMThreads)
       for (int v = 0; v < 4; ++v) part[gt * 16 + u * 4 + v] = acc[u][v];
   }
   __syncthreads();
-  if (grp == 1) return;
   const long long total = total_s;
   double* Mh = M + static_cast<size_t>(h) * d * d;
   const int jc[4] = {2 * tx, 2 * tx + 1, 32 + 2 * tx, 33 + 2 * tx};
+  if (gridDim.z == 1) {  // one slice: the block is complete
+    if (grp == 1) return;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int i = i0 + 4 * ty + u, j = j0 + jc[v];
+        const double sum = acc[u][v] + part[gt * 16 + u * 4 + v];
+        const double val = total > 0 ? sum / static_cast<double>(total) : (i == j ? 1.0 : 0.0);
+        Mh[static_cast<size_t>(i) * d + j] = val;
+        if (bi != bj) Mh[static_cast<size_t>(j) * d + i] = val;
+      }
+    return;
+  }
+  // this slice's partial block; the last slice to finish adds them all
+  const int blk = h * gridDim.x + blockIdx.x;
+  double* mine = mpart + (static_cast<size_t>(blk) * kMSplit + z) * (kMBlk * kMBlk);
+  if (grp == 0) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) mine[gt * 16 + u * 4 + v] = acc[u][v] + part[gt * 16 + u * 4 + v];
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last_s = atomicAdd(&mticket[blk], 1) == kMSplit - 1;
+  __syncthreads();
+  if (!last_s || grp == 1) return;
+  __threadfence();  // the other slices' partials are visible
+  if (threadIdx.x == 0) mticket[blk] = 0;  // ready for the next half-step
+  const double* all = mpart + static_cast<size_t>(blk) * kMSplit * (kMBlk * kMBlk);
 #pragma unroll
   for (int u = 0; u < 4; ++u)
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       const int i = i0 + 4 * ty + u, j = j0 + jc[v];
-      const double sum = acc[u][v] + part[gt * 16 + u * 4 + v];
+      double sum = 0.0;
+#pragma unroll
+      for (int zz = 0; zz < kMSplit; ++zz) sum += __ldcg(all + zz * (kMBlk * kMBlk) + gt * 16 + u * 4 + v);
       const double val = total > 0 ? sum / static_cast<double>(total) : (i == j ? 1.0 : 0.0);
       Mh[static_cast<size_t>(i) * d + j] = val;
       if (bi != bj) Mh[static_cast<size_t>(j) * d + i] = val;
@@ -201,15 +253,17 @@ __device__ __forceinline__ void kappa_parts(double kappa, bool real, uint16_t (&
 // nu_j = M mu_j and kappa_j = mu_j . nu_j in fp64; nu_j also as the pair of
 // bf16 rows nu_hi = bf16(nu_j), nu_lo = bf16(nu_j - nu_hi) that the scoring
 // MMA consumes (their sum is nu_j to 2^-18 relative), and |nu_j|. Clusters j
-// in [C, CP) are padding (nu = 0, kappa = +inf). grid (CP/32, BH), block 128:
-// warp w owns clusters j0 + 8w .. +7, lane owns dimensions 2 lane, 2 lane + 1
+// in [C, CP) are padding (nu = 0, kappa = +inf). grid (CP/kNuCl, BH), block
+// 128: warp w owns clusters j0 + 4w .. +3, lane owns dimensions 2 lane, 2 lane + 1
 // (and 64 + the same for d = 128). Rows of M arrive 16 at a time by cp.async,
 // one chunk ahead. M == nullptr means the identity. For the scoring MMA it
 // also writes, per head, the kappa parts tile (-kappa_j/2 in three bf16
 // parts, rows j of a [CP][16] tile in the no-swizzle core-matrix layout,
-// exactly as it lies in shared memory) and, per block of 32 clusters,
+// exactly as it lies in shared memory) and, per block of kNuCl clusters,
 // (max |nu_j|, max |kappa_j|) over its real clusters.
 constexpr int kNuRows = 16;
+constexpr int kNuCl = 16;            // clusters per block
+constexpr int kNuWarpCl = kNuCl / 4;  // clusters per warp
 constexpr int kExtraK = 16;  // K width of the kappa chunk of the scoring MMA
 constexpr int kNuMuStride = 130;  // doubles per staged centroid row (keeps 16-byte alignment)
 
@@ -228,9 +282,9 @@ __global__ void __launch_bounds__(128)
                      float2* __restrict__ numax) {
   extern __shared__ __align__(16) double nsm[];
   __shared__ float2 wmax[4];
-  double* mu = nsm;                          // [32][kNuMuStride]
-  double* mch = mu + 32 * kNuMuStride;       // two buffers of [16][d]
-  const int h = blockIdx.y, j0 = blockIdx.x * 32;
+  double* mu = nsm;                          // [kNuCl][kNuMuStride]
+  double* mch = mu + kNuCl * kNuMuStride;    // two buffers of [16][d]
+  const int h = blockIdx.y, j0 = blockIdx.x * kNuCl;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const double* Mh = M ? M + static_cast<size_t>(h) * d * d : nullptr;
   auto stage = [&](int chunk) {  // rows 16 chunk .. +15 of M into buffer chunk % 2
@@ -240,20 +294,20 @@ __global__ void __launch_bounds__(128)
     cp_async_commit();
   };
   if (Mh) stage(0);
-  {  // the block's 32 centroids, all float4 loads in flight before any store
-    constexpr int kLd = 32 * 128 / 4 / 128;  // float4 per thread (d = 128; half of them for d = 64)
+  {  // the block's centroids, all float4 loads in flight before any store
+    constexpr int kLd = kNuCl * 128 / 4 / 128;  // float4 per thread (d = 128; half of them for d = 64)
     float4 f[kLd];
 #pragma unroll
     for (int q = 0; q < kLd; ++q) {
       const int e = (threadIdx.x + q * 128) * 4, r = e / d, c = e % d;
       f[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < 32 * d && j0 + r < C)
+      if (e < kNuCl * d && j0 + r < C)
         f[q] = __ldg(reinterpret_cast<const float4*>(cent + (static_cast<size_t>(h) * C + j0 + r) * d + c));
     }
 #pragma unroll
     for (int q = 0; q < kLd; ++q) {
       const int e = (threadIdx.x + q * 128) * 4, r = e / d, c = e % d;
-      if (e < 32 * d) {
+      if (e < kNuCl * d) {
         double* m = mu + r * kNuMuStride + c;
         m[0] = f[q].x;
         m[1] = f[q].y;
@@ -264,10 +318,10 @@ __global__ void __launch_bounds__(128)
   }
   const int nd = d == 128 ? 4 : 2;  // dimensions per lane
   const int dim[4] = {2 * lane, 2 * lane + 1, 64 + 2 * lane, 65 + 2 * lane};
-  const double* mw = mu + 8 * warp * kNuMuStride;
-  double acc[8][4];  // [cluster][dimension]
+  const double* mw = mu + kNuWarpCl * warp * kNuMuStride;
+  double acc[kNuWarpCl][4];  // [cluster][dimension]
 #pragma unroll
-  for (int u = 0; u < 8; ++u)
+  for (int u = 0; u < kNuWarpCl; ++u)
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc[u][v] = 0.0;
   if (Mh) {
@@ -290,7 +344,7 @@ __global__ void __launch_bounds__(128)
         const double mv[4] = {m01.x, m01.y, m23.x, m23.y};
         const int li = ck * kNuRows + l;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < kNuWarpCl; ++u) {
           const double m_u = mw[u * kNuMuStride + li];
 #pragma unroll
           for (int v = 0; v < 4; ++v) acc[u][v] = fma(mv[v], m_u, acc[u][v]);
@@ -301,14 +355,14 @@ __global__ void __launch_bounds__(128)
   } else {
     __syncthreads();
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < kNuWarpCl; ++u)
 #pragma unroll
       for (int v = 0; v < 4; ++v) acc[u][v] = v < nd ? mw[u * kNuMuStride + dim[v]] : 0.0;
   }
   float mx_n = 0.f, mx_k = 0.f;
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int j = j0 + 8 * warp + u;
+  for (int u = 0; u < kNuWarpCl; ++u) {
+    const int j = j0 + kNuWarpCl * warp + u;
     double k1 = 0.0, k2 = 0.0;
     uint16_t hb[4], lb[4];
 #pragma unroll
@@ -364,10 +418,10 @@ __global__ void __launch_bounds__(128)
   if (threadIdx.x == 0) {
     float2 m = wmax[0];
     for (int w = 1; w < 4; ++w) m = make_float2(fmaxf(m.x, wmax[w].x), fmaxf(m.y, wmax[w].y));
-    numax[h * (CP / 32) + blockIdx.x] = m;
+    numax[h * (CP / kNuCl) + blockIdx.x] = m;
   }
 }
-inline size_t metric_nu_smem(int d) { return (32 * kNuMuStride + 2 * kNuRows * d) * sizeof(double); }
+inline size_t metric_nu_smem(int d) { return (kNuCl * kNuMuStride + 2 * kNuRows * d) * sizeof(double); }
 
 // ---------------------------------------------------------------- assign
 //
@@ -536,7 +590,7 @@ __device__ __forceinline__ void mark_ge(uint32_t& m, float v, float thr, uint32_
 // grid: min(#SMs, chunks) CTAs, block kAssignThreads. Dynamic smem:
 // [AssignSmem][X kStages x 128 x 64 bf16][nu_hi CP x D][nu_lo CP x D][ones 128 x 16][kappa parts CP x 16]
 // kimg: per head the kappa parts tile as it lies in shared memory; numax: per
-// head and 32-cluster block, (max |nu_j|, max |kappa_j|); xnorm: |x|^2 of the
+// head and kNuCl-cluster block, (max |nu_j|, max |kappa_j|); xnorm: |x|^2 of the
 // tokens (xnorm_kernel).
 template <int D, int CP>
 __global__ void __launch_bounds__(kAssignThreads, 1)
@@ -798,8 +852,8 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
         if (h != cur_h) {  // the head's bound maxima
           float mn = 0.f, mk = 0.f;
 #pragma unroll
-          for (int p = 0; p < CP / 32; ++p) {
-            const float2 m = __ldg(numax + h * (CP / 32) + p);
+          for (int p = 0; p < CP / kNuCl; ++p) {
+            const float2 m = __ldg(numax + h * (CP / kNuCl) + p);
             mn = fmaxf(mn, m.x);
             mk = fmaxf(mk, m.y);
           }
@@ -974,7 +1028,7 @@ __device__ __forceinline__ bool better(double sa, int ja, double sb, int jb) {
 }
 
 template <int D, int CP>
-__global__ void __launch_bounds__(kFixWarps * 32, 5)
+__global__ void __launch_bounds__(kFixWarps * 32, 8)
     fixup_kernel(const uint16_t* __restrict__ x, int N, int nv, int C, int BH, int ntiles,
                  const double* __restrict__ nu64, const double* __restrict__ kappa64,
                  int32_t* __restrict__ assign, const int32_t* __restrict__ defer_count,
@@ -1130,6 +1184,8 @@ __global__ void __launch_bounds__(kUpdThreads)
   __shared__ int dlt[kMaxClusters];   // count change per cluster
   __shared__ int base[kMaxClusters + 1];
   __shared__ uint16_t order[2 * kUpdTokens];
+  __shared__ uint16_t moved[kUpdTokens];  // incremental: the chunk's tokens whose label changed
+  __shared__ int n_moved;
   const int h = blockIdx.y, c0 = blockIdx.x * kUpdTokens;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (timed_out_before(err)) return;  // labels of an aborted step are not to be trusted
@@ -1137,8 +1193,26 @@ __global__ void __launch_bounds__(kUpdThreads)
   const int32_t* a = assign + static_cast<size_t>(h) * nv + c0;
   int32_t* pv = prev ? prev + static_cast<size_t>(h) * nv + c0 : nullptr;
   for (int j = tid; j < C; j += kUpdThreads) cnt[j] = dlt[j] = 0;
+  if (tid == 0) n_moved = 0;
   __syncthreads();
-  // a token's entries: (l, +) and, when it moved, (o, -); -1 for none
+  // incremental: list the moved tokens first (most did not move), so the two
+  // grouping passes below run over them only
+  if (pv) {
+    for (int t0 = warp * 32; t0 < n; t0 += kUpdThreads) {
+      const int t = t0 + lane;
+      const bool mv = t < n && a[t] != pv[t];
+      const unsigned bm = __ballot_sync(0xffffffffu, mv);
+      int at = 0;
+      if (lane == 0 && bm) at = atomicAdd(&n_moved, __popc(bm));
+      at = __shfl_sync(0xffffffffu, at, 0);
+      if (mv) moved[at + __popc(bm & ((1u << lane) - 1u))] = static_cast<uint16_t>(t);
+    }
+    __syncthreads();
+  }
+  const int n_items = pv ? n_moved : n;  // tokens the grouping passes visit
+  auto token_of = [&](int i) { return pv ? (i < n_items ? static_cast<int>(moved[i]) : n) : i; };
+  // a token's entries: (l, +) and, when it moved, (o, -); -1 for none (and
+  // for t = n, past the chunk)
   auto entries = [&](int t, int& l, int& o) {
     l = t < n ? a[t] : -1;
     o = -1;
@@ -1161,9 +1235,9 @@ __global__ void __launch_bounds__(kUpdThreads)
   // labels come in runs (neighbouring tokens share clusters): lanes with equal
   // labels add to the shared counters once, through their lowest lane
   const unsigned lt = (1u << lane) - 1u;
-  for (int t0 = warp * 32; t0 < n; t0 += kUpdThreads) {
+  for (int i0 = warp * 32; i0 < n_items; i0 += kUpdThreads) {
     int l, o;
-    entries(t0 + lane, l, o);
+    entries(token_of(i0 + lane), l, o);
     const unsigned pl = __match_any_sync(0xffffffffu, l);
     if (l >= 0 && (pl & lt) == 0) {
       atomicAdd(&cnt[l], __popc(pl));
@@ -1199,8 +1273,8 @@ __global__ void __launch_bounds__(kUpdThreads)
     cnt[j] = 0;
   }
   __syncthreads();
-  for (int t0 = warp * 32; t0 < n; t0 += kUpdThreads) {
-    const int t = t0 + lane;
+  for (int i0 = warp * 32; i0 < n_items; i0 += kUpdThreads) {
+    const int t = token_of(i0 + lane);
     int l, o;
     entries(t, l, o);
     const unsigned pl = __match_any_sync(0xffffffffu, l);
@@ -1316,6 +1390,8 @@ namespace {
 
 struct StepWs {
   double* M;
+  double* mpart;     // metric_m_kernel's partial blocks
+  int32_t* mticket;  // and their tickets (zero between launches)
   double* nu64;
   uint16_t* nu_hi;
   uint16_t* nu_lo;
@@ -1336,12 +1412,17 @@ struct StepWs {
 // per row read one or two 32-column TMEM chunks each
 inline int score_cols(int c) { return c <= 128 ? 128 : 256; }
 
-size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out) {
+// split_metric: metric_m_kernel in kMSplit slices with partial blocks (off for
+// the fixed-size scratch of the allocation-free entry point).
+size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out, bool split_metric = true) {
   Carver cv(ws);
   const int CP = score_cols(Cmax);
   const size_t ntiles = (static_cast<size_t>(nv) + kTileRows - 1) / kTileRows;
   StepWs w;
   w.M = cv.take<double>(static_cast<size_t>(BH) * d * d);
+  const int mblocks = (d / kMBlk) * (d / kMBlk + 1) / 2;
+  w.mpart = split_metric ? cv.take<double>(static_cast<size_t>(BH) * mblocks * kMSplit * kMBlk * kMBlk) : nullptr;
+  w.mticket = split_metric ? cv.take<int32_t>(static_cast<size_t>(BH) * mblocks) : nullptr;
   w.nu64 = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
   w.nu_hi = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * d);
   w.nu_lo = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * d);
@@ -1349,7 +1430,7 @@ size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out) {
   w.kappa = cv.take<float>(static_cast<size_t>(BH) * CP);
   w.nunorm = cv.take<float>(static_cast<size_t>(BH) * CP);
   w.kimg = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * kExtraK);
-  w.numax = cv.take<float2>(static_cast<size_t>(BH) * (CP / 32));
+  w.numax = cv.take<float2>(static_cast<size_t>(BH) * (CP / kNuCl));
   w.sums = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
   w.counts = cv.take<int32_t>(static_cast<size_t>(BH) * Cmax);
   w.head_next = cv.take<int32_t>(static_cast<size_t>(BH));
@@ -1445,7 +1526,9 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
   if (zero_C > 0) {
     if (cudaMemsetAsync(w.sums, 0, sizeof(double) * BH * static_cast<size_t>(zero_C) * d, st) != cudaSuccess ||
         cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * BH * static_cast<size_t>(zero_C), st) != cudaSuccess ||
-        cudaMemsetAsync(w.head_next, 0, sizeof(int32_t) * BH, st) != cudaSuccess)
+        cudaMemsetAsync(w.head_next, 0, sizeof(int32_t) * BH, st) != cudaSuccess ||
+        (w.mticket && cudaMemsetAsync(w.mticket, 0, sizeof(int32_t) * BH * (d / kMBlk) * (d / kMBlk + 1) / 2,
+                                      st) != cudaSuccess))
       return SVOO_ERR_CUDA;
   }
   if (metric_cent) {
@@ -1453,13 +1536,13 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
     if (cudaFuncSetAttribute(metric_m_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kMetricMSmem)) != cudaSuccess)
       return SVOO_ERR_CUDA;
-    metric_m_kernel<<<dim3(T * (T + 1) / 2, BH), kMThreads, kMetricMSmem, st>>>(metric_cent, metric_sizes,
-                                                                                metric_C, d, w.M);
+    metric_m_kernel<<<dim3(T * (T + 1) / 2, BH, w.mpart ? kMSplit : 1), kMThreads, kMetricMSmem, st>>>(
+        metric_cent, metric_sizes, metric_C, d, w.M, w.mpart, w.mticket);
   }
   if (cudaFuncSetAttribute(metric_nu_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(metric_nu_smem(d))) != cudaSuccess)
     return SVOO_ERR_CUDA;
-  metric_nu_kernel<<<dim3(CP / 32, BH), 128, metric_nu_smem(d), st>>>(
+  metric_nu_kernel<<<dim3(CP / kNuCl, BH), 128, metric_nu_smem(d), st>>>(
       metric_cent ? w.M : nullptr, cent, C, CP, d, w.nu64, w.nu_hi, w.nu_lo, w.kappa64, w.kappa,
       w.nunorm, w.kimg, w.numax);
   CUtensorMap xmap;
@@ -1646,13 +1729,13 @@ extern "C" svoo_status svoo_cluster_step_static(const svoo_shape* shape, const v
   if (!aligned(x, 16)) return SVOO_ERR_INVALID_ARG;
   const int BH = bh_of(shape);
   const int Cmax = step_clusters(C, metric_cent, metric_C);
-  if (carve_step(nullptr, BH, shape->d, Cmax, nvideo_of(shape), nullptr) > kStaticScratchBytes)
+  if (carve_step(nullptr, BH, shape->d, Cmax, nvideo_of(shape), nullptr, false) > kStaticScratchBytes)
     return SVOO_ERR_WORKSPACE;  // shape needs more than the fixed scratch holds
   int dev = 0;
   void* base = scratch_address(&dev);
   if (!base) return SVOO_ERR_CUDA;
   StepWs w;
-  carve_step(base, BH, shape->d, Cmax, nvideo_of(shape), &w);
+  carve_step(base, BH, shape->d, Cmax, nvideo_of(shape), &w, false);
   return run_step(shape, x, C, cent, sizes, assign, metric_cent, metric_sizes, metric_C, w, dev_err,
                   static_cast<cudaStream_t>(stream), C);
 }
