@@ -43,29 +43,24 @@ __global__ void init_centroids_kernel(const uint16_t* __restrict__ x, int N, int
 
 // ---------------------------------------------------------------- metric
 
-// M[h] = sum_b n_b c_b c_b^T / sum_b n_b in fp64. grid (T*(T+1)/2, BH,
-// kMSplit) with T = d/64 output blocks of 64 x 64 per side (upper triangle
-// only; an off-diagonal block is written to both (i, j) and (j, i), so M is
-// exactly symmetric); slice z of the grid sums the z-th quarter of the
-// clusters. Block 512 = two groups of 16 x 16 threads that take alternate
-// 32-cluster chunks of the slice; thread (ty, tx) of a group owns rows
-// i0 + 4ty .. +3 and columns j0 + {2tx, 2tx+1, 32+2tx, 33+2tx}. Each slice
-// writes its partial block (group 0's plus group 1's); the slice that
-// finishes last adds the kMSplit partials in slice order, so the result does
-// not depend on which slice ran when. The next chunk's values are fetched
-// into registers while the current one is used.
+// M[h] = sum_b n_b c_b c_b^T / sum_b n_b in fp64. grid (T*(T+1)/2, BH) with
+// T = d/64 output blocks of 64 x 64 per side (upper triangle only; an
+// off-diagonal block is written to both (i, j) and (j, i), so M is exactly
+// symmetric), block 512 = two groups of 16 x 16 threads that take alternate
+// 32-cluster chunks (their partial blocks are added at the end, group 0's
+// plus group 1's); thread (ty, tx) of a group owns rows i0 + 4ty .. +3 and
+// columns j0 + {2tx, 2tx+1, 32+2tx, 33+2tx}. The next chunk's values are
+// fetched into registers while the current one is used.
 constexpr int kMBlk = 64;
 constexpr int kMChunk = 32;
 constexpr int kMThreads = 512;
-constexpr int kMSplit = 4;
 
 __global__ void __launch_bounds__(kMThreads)
     metric_m_kernel(const float* __restrict__ cent, const int32_t* __restrict__ sizes, int C, int d,
-                    double* __restrict__ M, double* __restrict__ mpart, int32_t* __restrict__ mticket) {
+                    double* __restrict__ M) {
   extern __shared__ __align__(16) double msm[];   // per group: as[32][64], bs[32][64]
   __shared__ long long total_s;
-  __shared__ int last_s;
-  const int h = blockIdx.y, T = d / kMBlk, z = blockIdx.z;
+  const int h = blockIdx.y, T = d / kMBlk;
   int t = blockIdx.x, bi = 0;
   while (t >= T - bi) {  // upper-triangle block index -> (bi, bj), bi <= bj
     t -= T - bi;
@@ -103,26 +98,11 @@ __global__ void __launch_bounds__(kMThreads)
   for (int u = 0; u < 4; ++u)
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc[u][v] = 0.0;
-  // this slice's chunks: kc0 .. kc1 - 1
   const int nchunks = (C + kMChunk - 1) / kMChunk;
-  const int per = (nchunks + static_cast<int>(gridDim.z) - 1) / static_cast<int>(gridDim.z);
-  const int kc0 = min(nchunks, z * per), kc1 = min(nchunks, kc0 + per);
-  const int cend = min(C, kc1 * kMChunk);  // the slice's clusters end here
-  const int rounds = (kc1 - kc0 + 1) / 2;  // both groups run the same number of rounds
-  auto fetch_in = [&](int b0) {
-    if (b0 < cend) {
-      fetch(b0);
-    } else {
-#pragma unroll
-      for (int q = 0; q < kPer; ++q) {
-        fa[q] = fb[q] = 0.f;
-        nb_[q] = 0;
-      }
-    }
-  };
-  fetch_in((kc0 + grp) * kMChunk);
+  const int rounds = (nchunks + 1) / 2;  // both groups run the same number of rounds
+  fetch(grp * kMChunk);
   for (int rd = 0; rd < rounds; ++rd) {
-    const int b0 = (kc0 + 2 * rd + grp) * kMChunk;
+    const int b0 = (2 * rd + grp) * kMChunk;
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < kPer; ++q) {
@@ -131,8 +111,8 @@ __global__ void __launch_bounds__(kMThreads)
       bs[e] = static_cast<double>(fb[q]);
     }
     __syncthreads();
-    fetch_in(b0 + 2 * kMChunk);
-    const int nb = max(0, min(kMChunk, cend - b0));
+    if (b0 + 2 * kMChunk < C) fetch(b0 + 2 * kMChunk);
+    const int nb = max(0, min(kMChunk, C - b0));
     for (int bb = 0; bb < nb; ++bb) {
       const double2 a01 = *reinterpret_cast<const double2*>(&as[bb * kMBlk + 4 * ty]);
       const double2 a23 = *reinterpret_cast<const double2*>(&as[bb * kMBlk + 4 * ty + 2]);
@@ -162,48 +142,16 @@ __global__ void __launch_bounds__(kMThreads)
       for (int v = 0; v < 4; ++v) part[gt * 16 + u * 4 + v] = acc[u][v];
   }
   __syncthreads();
+  if (grp == 1) return;
   const long long total = total_s;
   double* Mh = M + static_cast<size_t>(h) * d * d;
   const int jc[4] = {2 * tx, 2 * tx + 1, 32 + 2 * tx, 33 + 2 * tx};
-  if (gridDim.z == 1) {  // one slice: the block is complete
-    if (grp == 1) return;
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const int i = i0 + 4 * ty + u, j = j0 + jc[v];
-        const double sum = acc[u][v] + part[gt * 16 + u * 4 + v];
-        const double val = total > 0 ? sum / static_cast<double>(total) : (i == j ? 1.0 : 0.0);
-        Mh[static_cast<size_t>(i) * d + j] = val;
-        if (bi != bj) Mh[static_cast<size_t>(j) * d + i] = val;
-      }
-    return;
-  }
-  // this slice's partial block; the last slice to finish adds them all
-  const int blk = h * gridDim.x + blockIdx.x;
-  double* mine = mpart + (static_cast<size_t>(blk) * kMSplit + z) * (kMBlk * kMBlk);
-  if (grp == 0) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) mine[gt * 16 + u * 4 + v] = acc[u][v] + part[gt * 16 + u * 4 + v];
-  }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last_s = atomicAdd(&mticket[blk], 1) == kMSplit - 1;
-  __syncthreads();
-  if (!last_s || grp == 1) return;
-  __threadfence();  // the other slices' partials are visible
-  if (threadIdx.x == 0) mticket[blk] = 0;  // ready for the next half-step
-  const double* all = mpart + static_cast<size_t>(blk) * kMSplit * (kMBlk * kMBlk);
 #pragma unroll
   for (int u = 0; u < 4; ++u)
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
       const int i = i0 + 4 * ty + u, j = j0 + jc[v];
-      double sum = 0.0;
-#pragma unroll
-      for (int zz = 0; zz < kMSplit; ++zz) sum += __ldcg(all + zz * (kMBlk * kMBlk) + gt * 16 + u * 4 + v);
+      const double sum = acc[u][v] + part[gt * 16 + u * 4 + v];
       const double val = total > 0 ? sum / static_cast<double>(total) : (i == j ? 1.0 : 0.0);
       Mh[static_cast<size_t>(i) * d + j] = val;
       if (bi != bj) Mh[static_cast<size_t>(j) * d + i] = val;
@@ -1390,8 +1338,6 @@ namespace {
 
 struct StepWs {
   double* M;
-  double* mpart;     // metric_m_kernel's partial blocks
-  int32_t* mticket;  // and their tickets (zero between launches)
   double* nu64;
   uint16_t* nu_hi;
   uint16_t* nu_lo;
@@ -1412,17 +1358,12 @@ struct StepWs {
 // per row read one or two 32-column TMEM chunks each
 inline int score_cols(int c) { return c <= 128 ? 128 : 256; }
 
-// split_metric: metric_m_kernel in kMSplit slices with partial blocks (off for
-// the fixed-size scratch of the allocation-free entry point).
-size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out, bool split_metric = true) {
+size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out) {
   Carver cv(ws);
   const int CP = score_cols(Cmax);
   const size_t ntiles = (static_cast<size_t>(nv) + kTileRows - 1) / kTileRows;
   StepWs w;
   w.M = cv.take<double>(static_cast<size_t>(BH) * d * d);
-  const int mblocks = (d / kMBlk) * (d / kMBlk + 1) / 2;
-  w.mpart = split_metric ? cv.take<double>(static_cast<size_t>(BH) * mblocks * kMSplit * kMBlk * kMBlk) : nullptr;
-  w.mticket = split_metric ? cv.take<int32_t>(static_cast<size_t>(BH) * mblocks) : nullptr;
   w.nu64 = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
   w.nu_hi = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * d);
   w.nu_lo = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * d);
@@ -1526,9 +1467,7 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
   if (zero_C > 0) {
     if (cudaMemsetAsync(w.sums, 0, sizeof(double) * BH * static_cast<size_t>(zero_C) * d, st) != cudaSuccess ||
         cudaMemsetAsync(w.counts, 0, sizeof(int32_t) * BH * static_cast<size_t>(zero_C), st) != cudaSuccess ||
-        cudaMemsetAsync(w.head_next, 0, sizeof(int32_t) * BH, st) != cudaSuccess ||
-        (w.mticket && cudaMemsetAsync(w.mticket, 0, sizeof(int32_t) * BH * (d / kMBlk) * (d / kMBlk + 1) / 2,
-                                      st) != cudaSuccess))
+        cudaMemsetAsync(w.head_next, 0, sizeof(int32_t) * BH, st) != cudaSuccess)
       return SVOO_ERR_CUDA;
   }
   if (metric_cent) {
@@ -1536,8 +1475,8 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
     if (cudaFuncSetAttribute(metric_m_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kMetricMSmem)) != cudaSuccess)
       return SVOO_ERR_CUDA;
-    metric_m_kernel<<<dim3(T * (T + 1) / 2, BH, w.mpart ? kMSplit : 1), kMThreads, kMetricMSmem, st>>>(
-        metric_cent, metric_sizes, metric_C, d, w.M, w.mpart, w.mticket);
+    metric_m_kernel<<<dim3(T * (T + 1) / 2, BH), kMThreads, kMetricMSmem, st>>>(metric_cent, metric_sizes,
+                                                                                metric_C, d, w.M);
   }
   if (cudaFuncSetAttribute(metric_nu_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(metric_nu_smem(d))) != cudaSuccess)
@@ -1729,13 +1668,13 @@ extern "C" svoo_status svoo_cluster_step_static(const svoo_shape* shape, const v
   if (!aligned(x, 16)) return SVOO_ERR_INVALID_ARG;
   const int BH = bh_of(shape);
   const int Cmax = step_clusters(C, metric_cent, metric_C);
-  if (carve_step(nullptr, BH, shape->d, Cmax, nvideo_of(shape), nullptr, false) > kStaticScratchBytes)
+  if (carve_step(nullptr, BH, shape->d, Cmax, nvideo_of(shape), nullptr) > kStaticScratchBytes)
     return SVOO_ERR_WORKSPACE;  // shape needs more than the fixed scratch holds
   int dev = 0;
   void* base = scratch_address(&dev);
   if (!base) return SVOO_ERR_CUDA;
   StepWs w;
-  carve_step(base, BH, shape->d, Cmax, nvideo_of(shape), &w, false);
+  carve_step(base, BH, shape->d, Cmax, nvideo_of(shape), &w);
   return run_step(shape, x, C, cent, sizes, assign, metric_cent, metric_sizes, metric_C, w, dev_err,
                   static_cast<cudaStream_t>(stream), C);
 }
