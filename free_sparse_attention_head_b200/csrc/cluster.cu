@@ -6,9 +6,9 @@
 //
 // Kernels of one half-step (one side):
 //   metric_m_kernel   M from the other side's centroids and sizes (fp64)
-//   metric_nu_kernel  nu_j = M mu_j, kappa_j = mu_j . nu_j (fp64), |nu_j|,
-//                     nu_j split into two bf16 rows (hi + lo), -kappa_j/2 in
-//                     three bf16 parts, and per-block maxima for the bound
+//   metric_nu_kernel  nu_j = M mu_j, kappa_j = mu_j . nu_j (fp64), nu_j split
+//                     into two bf16 rows (hi + lo), -kappa_j/2 in three bf16
+//                     parts, and per-block maxima of |nu_j|, |kappa_j| for the bound
 //   xnorm_kernel      |x|^2 of every token, once per side and call (the
 //                     assignment's error bound)
 //   assign_kernel     persistent, warp-specialised, dynamically scheduled
@@ -200,7 +200,7 @@ __device__ __forceinline__ void kappa_parts(double kappa, bool real, uint16_t (&
 
 // nu_j = M mu_j and kappa_j = mu_j . nu_j in fp64; nu_j also as the pair of
 // bf16 rows nu_hi = bf16(nu_j), nu_lo = bf16(nu_j - nu_hi) that the scoring
-// MMA consumes (their sum is nu_j to 2^-18 relative), and |nu_j|. Clusters j
+// MMA consumes (their sum is nu_j to 2^-18 relative). Clusters j
 // in [C, CP) are padding (nu = 0, kappa = +inf). grid (CP/kNuCl, BH), block
 // 128: warp w owns clusters j0 + 4w .. +3, lane owns dimensions 2 lane, 2 lane + 1
 // (and 64 + the same for d = 128). Rows of M arrive 16 at a time by cp.async,
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(128)
     metric_nu_kernel(const double* __restrict__ M, const float* __restrict__ cent, int C, int CP,
                      int d, double* __restrict__ nu64, uint16_t* __restrict__ nu_hi,
                      uint16_t* __restrict__ nu_lo, double* __restrict__ kappa64,
-                     float* __restrict__ kappa32, float* __restrict__ nunorm, uint16_t* __restrict__ kimg,
+                     uint16_t* __restrict__ kimg,
                      float2* __restrict__ numax) {
   extern __shared__ __align__(16) double nsm[];
   __shared__ float2 wmax[4];
@@ -347,8 +347,6 @@ __global__ void __launch_bounds__(128)
     if (lane == 0) {
       const float nn = j < C ? static_cast<float>(sqrt(k2)) : 0.f;
       kappa64[h * CP + j] = j < C ? k1 : INFINITY;
-      kappa32[h * CP + j] = j < C ? static_cast<float>(k1) : INFINITY;
-      nunorm[h * CP + j] = nn;
       uint16_t p[3];
       kappa_parts(k1, j < C, p);
       uint8_t* img = reinterpret_cast<uint8_t*>(kimg + static_cast<size_t>(h) * CP * kExtraK);
@@ -1342,8 +1340,6 @@ struct StepWs {
   uint16_t* nu_hi;
   uint16_t* nu_lo;
   double* kappa64;
-  float* kappa;
-  float* nunorm;
   uint16_t* kimg;
   float2* numax;
   double* sums;
@@ -1368,8 +1364,6 @@ size_t carve_step(void* ws, int BH, int d, int Cmax, int nv, StepWs* out) {
   w.nu_hi = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * d);
   w.nu_lo = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * d);
   w.kappa64 = cv.take<double>(static_cast<size_t>(BH) * CP);
-  w.kappa = cv.take<float>(static_cast<size_t>(BH) * CP);
-  w.nunorm = cv.take<float>(static_cast<size_t>(BH) * CP);
   w.kimg = cv.take<uint16_t>(static_cast<size_t>(BH) * CP * kExtraK);
   w.numax = cv.take<float2>(static_cast<size_t>(BH) * (CP / kNuCl));
   w.sums = cv.take<double>(static_cast<size_t>(BH) * Cmax * d);
@@ -1482,8 +1476,8 @@ svoo_status run_step(const svoo_shape* sh, const void* x, int C, float* cent, in
                            static_cast<int>(metric_nu_smem(d))) != cudaSuccess)
     return SVOO_ERR_CUDA;
   metric_nu_kernel<<<dim3(CP / kNuCl, BH), 128, metric_nu_smem(d), st>>>(
-      metric_cent ? w.M : nullptr, cent, C, CP, d, w.nu64, w.nu_hi, w.nu_lo, w.kappa64, w.kappa,
-      w.nunorm, w.kimg, w.numax);
+      metric_cent ? w.M : nullptr, cent, C, CP, d, w.nu64, w.nu_hi, w.nu_lo, w.kappa64, w.kimg,
+      w.numax);
   CUtensorMap xmap;
   if (encode_tiled_2d(&xmap, x, static_cast<uint64_t>(BH) * N, d, kTileRows, 64) != CUDA_SUCCESS)
     return SVOO_ERR_CUDA;
