@@ -907,12 +907,13 @@ __global__ void __launch_bounds__(kAssignThreads, 1)
 template <int D>
 __device__ __forceinline__ double exact_score(const uint16_t* __restrict__ xrow, const double* __restrict__ nj,
                                               double kap_j) {
-  // sixteen independent fp64 FMA chains, summed pairwise: an fp64 FMA's
-  // dependent latency is long on this GPU, so short chains matter more than
-  // the instruction count
-  double e[16];
+  // eight independent fp64 FMA chains, summed pairwise: an fp64 FMA's
+  // dependent latency is long on this GPU, so short chains matter; eight
+  // (not sixteen) leave registers for 12 blocks of fixup_kernel per SM, which
+  // measured faster
+  double e[8];
 #pragma unroll
-  for (int u = 0; u < 16; ++u) e[u] = 0.0;
+  for (int u = 0; u < 8; ++u) e[u] = 0.0;
 #pragma unroll 2
   for (int i = 0; i < D; i += 16) {
     const uint4 xa = __ldg(reinterpret_cast<const uint4*>(xrow + i));
@@ -921,12 +922,12 @@ __device__ __forceinline__ double exact_score(const uint16_t* __restrict__ xrow,
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const double2 nv = __ldg(reinterpret_cast<const double2*>(nj + i + 2 * u));
-      e[2 * u] = fma(static_cast<double>(__uint_as_float(w[u] << 16)), nv.x, e[2 * u]);
-      e[2 * u + 1] = fma(static_cast<double>(__uint_as_float(w[u] & 0xffff0000u)), nv.y, e[2 * u + 1]);
+      e[u] = fma(static_cast<double>(__uint_as_float(w[u] << 16)), nv.x, e[u]);
+      e[u] = fma(static_cast<double>(__uint_as_float(w[u] & 0xffff0000u)), nv.y, e[u]);
     }
   }
 #pragma unroll
-  for (int step = 8; step > 0; step >>= 1)
+  for (int step = 4; step > 0; step >>= 1)
 #pragma unroll
     for (int u = 0; u < step; ++u) e[u] += e[u + step];
   return kap_j - 2.0 * e[0];
@@ -966,7 +967,8 @@ __device__ int decide_all(const uint16_t* __restrict__ xrow, const double* __res
 // over the lanes of each row's run (ties to the smaller j) goes to the row's
 // own lane, which keeps the row's best over the rounds. Rows labelled -2 (by
 // the scorers, or here for a list that does not look right): the whole warp
-// compares every cluster (decide_all).
+// compares every cluster (decide_all). 12 blocks per SM: more warps in flight
+// hide the fp64 latency better than spill-free registers did.
 constexpr int kFixWarps = 4;
 
 __device__ __forceinline__ bool better(double sa, int ja, double sb, int jb) {
@@ -974,7 +976,7 @@ __device__ __forceinline__ bool better(double sa, int ja, double sb, int jb) {
 }
 
 template <int D, int CP>
-__global__ void __launch_bounds__(kFixWarps * 32, 8)
+__global__ void __launch_bounds__(kFixWarps * 32, 12)
     fixup_kernel(const uint16_t* __restrict__ x, int N, int nv, int C, int BH, int ntiles,
                  const double* __restrict__ nu64, const double* __restrict__ kappa64,
                  int32_t* __restrict__ assign, const int32_t* __restrict__ defer_count,
