@@ -19,9 +19,12 @@
 //   fixup_kernel      the other tokens, exactly in fp64: their listed
 //                     candidates, or every cluster (ties to the smaller j)
 //   update_kernel     member sums in fp64, exact (so order-independent), per
-//                     chunk of consecutive tokens grouped by label
+//                     chunk of consecutive tokens grouped by label; within a
+//                     call, after each side's first half-step, only the tokens
+//                     whose label changed move between the kept sums
 //   finalize_kernel   centroid = fp32(sum / count), empty clusters keep
-//                     theirs; resets the sums for the next half-step.
+//                     theirs; resets the chunk counters (and a lone
+//                     half-step's sums).
 #include <math.h>
 
 #include "common.cuh"
