@@ -95,9 +95,10 @@ def _launch_count(iters, psa=False):
     # psa: labels + mask 2; permute 5 (sort, tiles, 3 gathers); attention 1
     if psa:
         return 2 + 5 + 1
-    # init x2; round 0: q (nu, assign, finalize) + k (m, nu, assign, finalize);
-    # later rounds 4 + 4; mask 3; permute 5; attention 1
-    return 2 + 7 + 8 * (iters - 1) + 3 + 5 + 1
+    # cold co-clustering call: init x2, |x|^2 x2; round 0: q (nu, assign, fixup,
+    # update, finalize) + k (m and the same five); later rounds 6 + 6; mask 3
+    # (pair mass, select, tail merge); permute 5; attention 1
+    return 2 + 2 + 5 + 6 + 12 * (iters - 1) + 3 + 5 + 1
 
 
 class ClockSampler:
